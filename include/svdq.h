@@ -1,0 +1,173 @@
+/*
+ * svdq.h — C ABI of the SVDQuant W4A4 linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer (devpress.csdn.net SVDQuant paper walkthrough, eq. (5)):
+ *
+ *     X W  =  X_hat W_hat  ~=  (X_hat L1) L2  +  Q(X_hat) Q(R)
+ *
+ *   X_hat = X diag(lambda)^-1                smoothed activation
+ *   W_hat = diag(lambda) W = L1 L2 + R       16-bit rank-r branch + residual
+ *   Q(.)  = NVFP4: E2M1 codes, one E4M3 scale per 16 K-elements (eq. (1), q_max = 6)
+ *
+ * Conventions used by every entry point:
+ *
+ *   Orientation.  X is [M][K] (M tokens, K input channels). The weight is given
+ *     in nn.Linear orientation W_lin [N][K]; the paper's W is W_lin^T. Y is [M][N].
+ *   Memory.  Every pointer is a DEVICE pointer to memory the caller owns, aligned
+ *     to 16 bytes (SVDQ_ERR_MISALIGNED otherwise). The library allocates nothing
+ *     on the per-call path; svdq_prepare_weights works inside the caller's
+ *     workspace. All matrices are dense row-major with no padding between rows.
+ *   Streams.  `stream` is a cudaStream_t (NULL = legacy default stream). Calls
+ *     are asynchronous with respect to the host unless stated otherwise.
+ *   Shapes.  M >= 0 (M == 0 is a no-op), K >= 128 and K % 128 == 0,
+ *     N >= 128 and N % 128 == 0, rank % 16 == 0 and 0 <= rank <= 128;
+ *     anything else returns SVDQ_ERR_UNSUPPORTED_SHAPE.
+ *   Errors.  No entry point aborts or throws. Launch failures return
+ *     SVDQ_ERR_CUDA (details in svdq_last_error()). A kernel that gives up on a
+ *     bounded wait records a device error word; svdq_check() reads it
+ *     (SVDQ_ERR_TIMEOUT) and clears it.
+ *   Device.  A device other than compute capability 10.0 returns
+ *     SVDQ_ERR_NO_DEVICE. There is no CPU fallback.
+ *
+ * Buffer formats (byte sizes come from svdq_act_sizes / svdq_weight_sizes):
+ *
+ *   codes   uint8 [rows][K/2]: E2M1 nibbles, element 2i in the low nibble.
+ *   scales  E4M3 bytes in the native tile layout: for row block rb (128 rows)
+ *           and K block kb (64 elements) a 512-byte atom at offset
+ *           (rb * K/64 + kb) * 512; inside it, row 32q + i and group j (0..3)
+ *           of the block sit at byte 16*i + 4*q + j. Rows past the end of the
+ *           matrix hold zero. svdq_scales_to_canonical() gives [rows][K/16].
+ *   L1p     bf16 [rank][K]: the down-projection factor with the smoothing folded
+ *           in, L1p[k][j] = bf16(L1[j][k] / lambda_j), so that X L1p^T == X_hat L1.
+ *   L2t     bf16 [N][rank]: the up-projection factor, L2t[n][k] = bf16(L2[k][n]).
+ *   T       bf16 [M][rank]: the down-projection X_hat L1.
+ */
+#ifndef SVDQ_H_
+#define SVDQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,        /* null pointer where one is required, bad enum, alpha out of range */
+  SVDQ_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the conventions above */
+  SVDQ_ERR_MISALIGNED = 3,         /* a pointer is not 16-byte aligned */
+  SVDQ_ERR_BUFFER_TOO_SMALL = 4,   /* workspace smaller than svdq_weight_sizes() asks for */
+  SVDQ_ERR_NO_DEVICE = 5,          /* no CUDA device, or not compute capability 10.0 */
+  SVDQ_ERR_CUDA = 6,               /* a CUDA runtime call or kernel launch failed */
+  SVDQ_ERR_TIMEOUT = 7,            /* a kernel gave up on a bounded wait (see svdq_check) */
+  SVDQ_ERR_INTERNAL = 8
+} svdq_status;
+
+typedef enum {
+  SVDQ_FUSED = 0,    /* low-rank down-projection inside the quantize pass, up-projection
+                        inside the 4-bit GEMM's accumulator (walkthrough Fig. 6) */
+  SVDQ_UNFUSED = 1   /* the same arithmetic as separate passes: the down-projection
+                        re-reads X, the up-projection re-reads and re-writes Y */
+} svdq_variant;
+
+/* Problem shape. The quantization group is fixed at 16. */
+typedef struct {
+  int64_t M;
+  int64_t K;
+  int64_t N;
+  int32_t rank;
+} svdq_shape;
+
+/* Flags of svdq_prepare_weights. */
+#define SVDQ_PREPARE_GIVEN_FACTORS 1u  /* L1p and L2t are inputs: use the caller's factors */
+
+/* Human-readable name of a status code (static storage; never NULL). */
+SVDQ_API const char* svdq_status_string(int status);
+
+/* Last error message of the calling host thread (static thread-local storage). */
+SVDQ_API const char* svdq_last_error(void);
+
+/* Library ABI version: 100 * major + minor. */
+SVDQ_API int svdq_version(void);
+
+/* Byte sizes of the per-call buffers for `shape`: codes Qx, native scales Sx,
+ * and T (0 when rank == 0). Any output pointer may be NULL. Host only. */
+SVDQ_API svdq_status svdq_act_sizes(svdq_shape shape, size_t* qx_bytes, size_t* sx_bytes, size_t* t_bytes);
+
+/* Byte sizes of the prepared-weight buffers (Qr codes, native Sr scales, L1p,
+ * L2t) and of the workspace svdq_prepare_weights needs. Any output pointer may
+ * be NULL. Host only. */
+SVDQ_API svdq_status svdq_weight_sizes(svdq_shape shape, size_t* qr_bytes, size_t* sr_bytes, size_t* l1p_bytes,
+                              size_t* l2t_bytes, size_t* workspace_bytes);
+
+/* Per-channel activation maximum for the smoothing rule (calibration):
+ * amax[j] = max_m |X[m][j]|. X bf16 [M][K], amax fp32 [K] (overwritten).
+ * K % 8 == 0 suffices here; M >= 1.
+ * (anrans.github.io AI-infra handbook, Quantization chapter, SmoothQuant.) */
+SVDQ_API svdq_status svdq_channel_amax(int64_t M, int64_t K, const void* X, float* amax, void* stream);
+
+/* Offline weight preparation (not on the per-call path):
+ *   1. smoothing factors: lambda_j = amax_j^alpha / max_n|W_lin[n][j]|^(1-alpha),
+ *      lambda_j = 1 where either maximum is 0; lambda = fp32(.), inv_lambda =
+ *      fp32(1/lambda)  (handbook SmoothQuant section);
+ *   2. W_hat = diag(lambda) W_lin^T and its top-rank SVD split W_hat ~= L1 L2 with
+ *      the singular values in L1 (walkthrough: SVD paragraph after eq. (8);
+ *      handbook SVDQuant section). Without SVDQ_PREPARE_GIVEN_FACTORS the library
+ *      computes it (randomized subspace iteration in fp64 on the device) and
+ *      writes L1p and L2t; with it, L1p and L2t are read as given;
+ *   3. residual R = fp32(W_hat - sum_k (lambda * L1p[k]) L2t[:,k]) in fp64, in
+ *      increasing k, no fused multiply-add (eq. (5));
+ *   4. NVFP4 encoding of R grouped along K: codes Qr [N][K/2], native scales Sr.
+ * W_lin bf16 [N][K]; act_amax fp32 [K]; alpha in [0, 1]; lambda, inv_lambda fp32
+ * [K] (written); workspace of at least svdq_weight_sizes()'s workspace_bytes
+ * (may be NULL when that size is 0). Stream-ordered; the caller's buffers are
+ * ready when the stream reaches the end of the call. */
+SVDQ_API svdq_status svdq_prepare_weights(svdq_shape shape, const void* W_lin, const float* act_amax, float alpha,
+                                 unsigned int flags, void* L1p, void* L2t, void* Qr, void* Sr,
+                                 float* lambda, float* inv_lambda, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
+/* Per-call activation quantization with the low-rank down-projection.
+ * X bf16 [M][K]; inv_lambda fp32 [K]; L1p bf16 [rank][K].
+ * Writes Qx codes [M][K/2], Sx native scales, T bf16 [M][rank]:
+ *   x_hat = fp32(fp32(x) * inv_lambda[k]);
+ *   per 16-group: s = E4M3_rne_satfinite(fp32(max|x_hat| / 6)),
+ *                 q = E2M1_rne_satfinite(fp32(x_hat * fp32(1/s))), all +0 if s == 0;
+ *   T = bf16(X L1p^T)  (fp32 accumulation)
+ * (eq. (1), Table 3's NVFP4 microscaling, Fig. 6's fused down-projection).
+ * variant SVDQ_FUSED reads X once; SVDQ_UNFUSED runs the down-projection as a
+ * second pass over X. rank == 0: L1p and T may be NULL. */
+SVDQ_API svdq_status svdq_quantize_act(svdq_shape shape, const void* X, const float* inv_lambda, const void* L1p,
+                              void* Qx, void* Sx, void* T, int variant, void* stream);
+
+/* Per-call W4A4 GEMM with the low-rank up-projection:
+ *   Y = bf16( deq(Qx) deq(Qr)^T + T L2t^T )   (fp32 accumulation)
+ * (eq. (2), eq. (5)). Qx/Sx as written by svdq_quantize_act, Qr/Sr/L2t as
+ * written by svdq_prepare_weights, Y bf16 [M][N]. variant SVDQ_FUSED adds T L2
+ * into the GEMM's tensor-memory accumulator; SVDQ_UNFUSED runs the GEMM with
+ * no branch, then a second kernel reads Y, adds T L2 in fp32 and writes Y.
+ * rank == 0: T and L2t may be NULL. */
+SVDQ_API svdq_status svdq_linear(svdq_shape shape, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                        const void* Sr, const void* L2t, void* Y, int variant, void* stream);
+
+/* Native scale layout -> canonical [rows][K/16] bytes (inspection helper). */
+SVDQ_API svdq_status svdq_scales_to_canonical(int64_t rows, int64_t K, const void* native, void* canonical,
+                                     void* stream);
+
+/* Synchronize `stream`, then read and clear the device error word of the
+ * current device. Returns SVDQ_ERR_TIMEOUT if a kernel gave up on a bounded
+ * wait since the last check, SVDQ_ERR_CUDA on an asynchronous CUDA error. */
+SVDQ_API svdq_status svdq_check(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H_ */

@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/svdq.h declares, answers size queries, and rejects bad
+shapes, null and misaligned pointers with the documented status codes before
+touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from w4a4_diffusion_model_b200 import build as B
+from w4a4_diffusion_model_b200 import svdq as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return S.load()
+
+
+def header_symbols():
+    with open(os.path.join(ROOT, "include", "svdq.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"SVDQ_API\s+[\w\s\*]+?\b(svdq_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    syms = header_symbols()
+    assert len(syms) >= 11
+    for s in syms:
+        assert hasattr(lib, s), s
+    assert set(syms) == set(S.EXPORTS)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.svdq_version() == 100
+    for code, name in S.STATUS.items():
+        assert lib.svdq_status_string(code).decode() == name
+    assert lib.svdq_status_string(99).decode() == "SVDQ_ERR_UNKNOWN"
+
+
+def test_size_queries():
+    qx, sx, t = S.svdq_act_sizes(S.LayerShape(4608, 3072, 12288, 32))
+    assert qx == 4608 * 1536 and sx == 36 * 48 * 512 and t == 4608 * 32 * 2
+    qx, sx, t = S.svdq_act_sizes(S.LayerShape(130, 384, 128, 0))
+    assert qx == 130 * 192 and sx == 2 * 6 * 512 and t == 0
+    qr, sr, l1, l2, ws = S.svdq_weight_sizes(S.LayerShape(0, 12288, 3072, 32))
+    assert qr == 3072 * 6144 and sr == 24 * 192 * 512 and l1 == 32 * 12288 * 2 and l2 == 3072 * 32 * 2
+    assert ws >= 0
+
+
+@pytest.mark.parametrize("M,K,N,r", [(-1, 128, 128, 0), (1, 100, 128, 0), (1, 128, 100, 0), (1, 128, 128, 8),
+                                     (1, 128, 128, 144), (1, 64, 128, 16), (1, 128, 128, -16)])
+def test_bad_shapes_rejected(lib, M, K, N, r):
+    sh = S.Shape(M, K, N, r)
+    a = ctypes.c_size_t()
+    assert lib.svdq_act_sizes(sh, ctypes.byref(a), None, None) == 2
+    assert lib.svdq_quantize_act(sh, None, None, None, None, None, None, 0, None) == 2
+    assert lib.svdq_linear(sh, None, None, None, None, None, None, None, 0, None) == 2
+
+
+def test_null_misaligned_and_variant_rejected(lib):
+    sh = S.Shape(128, 256, 128, 16)
+    good = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    assert lib.svdq_quantize_act(sh, good, good, good, good, good, None, 0, None) == 1          # T missing
+    assert lib.svdq_quantize_act(sh, good, good, good, good, good, good, 7, None) == 1         # variant
+    assert lib.svdq_quantize_act(sh, good, good, good, bad, good, good, 0, None) == 3          # misaligned
+    assert lib.svdq_linear(sh, good, good, good, good, good, bad, good, 0, None) == 3
+    assert lib.svdq_linear(sh, good, good, None, good, good, good, good, 0, None) == 1
+    assert lib.svdq_prepare_weights(sh, good, good, ctypes.c_float(1.5), 0, good, good, good, good, good, good,
+                                    None, 0, None) == 1                                         # alpha
+    assert lib.svdq_prepare_weights(sh, good, good, ctypes.c_float(0.5), 4, good, good, good, good, good, good,
+                                    None, 0, None) == 1                                         # flags
+    assert lib.svdq_channel_amax(0, 128, good, good, None) == 2
+    assert lib.svdq_channel_amax(4, 128, good, bad, None) == 3
+    assert b"aligned" in lib.svdq_last_error()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_is_reported_not_emulated(lib):
+    sh = S.Shape(128, 256, 128, 0)
+    good = ctypes.c_void_p(1 << 20)
+    assert lib.svdq_quantize_act(sh, good, good, None, good, good, None, 0, None) == 5
+    assert lib.svdq_linear(sh, good, good, None, good, good, None, good, 0, None) == 5
+    assert lib.svdq_check(None) == 5

@@ -1,0 +1,415 @@
+// C ABI of the SVDQuant W4A4 linear layer (declared in include/svdq.h):
+// argument checks, tensor-map construction and kernel launches. The kernels
+// live in the headers included below; this file is the library's single
+// translation unit.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "svdq.h"
+#include "svdq_gemm.cuh"
+#include "svdq_prepare.cuh"
+#include "svdq_quant.cuh"
+#include "svdq_svd.cuh"
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+}
+
+svdq_status fail(svdq_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+#define SVDQ_CUDA(call)                                                                           \
+  do {                                                                                            \
+    cudaError_t e_ = (call);                                                                      \
+    if (e_ != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_));   \
+  } while (0)
+
+#define SVDQ_LAUNCHED(what)                                                                       \
+  do {                                                                                            \
+    cudaError_t e_ = cudaGetLastError();                                                          \
+    if (e_ != cudaSuccess) return fail(SVDQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e_));    \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+svdq_status check_shape(const svdq_shape& s) {
+  if (s.M < 0 || s.K < 128 || s.N < 128 || s.K % 128 || s.N % 128 || s.rank < 0 || s.rank > 128 ||
+      s.rank % 16)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE,
+                "shape M=%lld K=%lld N=%lld rank=%d: need M>=0, K,N multiples of 128, rank in {0,16,...,128}",
+                (long long)s.M, (long long)s.K, (long long)s.N, (int)s.rank);
+  if (s.M > (1ll << 31) - 1 || s.K > (1ll << 20) || s.N > (1ll << 24))
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "shape too large for 32-bit tile coordinates");
+  return SVDQ_OK;
+}
+
+// Device check (compute capability 10.0), cached per device ordinal.
+svdq_status check_device() {
+  static std::mutex mu;
+  static int cached[64];   // 0 unknown, 1 ok, 2 bad
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return fail(SVDQ_ERR_NO_DEVICE, "no CUDA device");
+  }
+  if (dev < 64) {
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[dev] == 0) {
+      int major = 0, minor = 0;
+      if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+          cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SVDQ_ERR_NO_DEVICE, "cannot query device %d", dev);
+      }
+      cached[dev] = (major == 10 && minor == 0) ? 1 : 2;
+    }
+    if (cached[dev] != 1) return fail(SVDQ_ERR_NO_DEVICE, "device %d is not compute capability 10.0 (sm_100a)", dev);
+  }
+  return SVDQ_OK;
+}
+
+// ---------------------------------------------------------------- tensor maps
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [rows][cols] of `elem_bytes`-sized elements, box of
+// box_cols x box_rows, zero fill out of bounds.
+svdq_status make_tmap(CUtensorMap* tm, const void* base, CUtensorMapDataType dt, int elem_bytes, uint64_t cols,
+                      uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * (uint64_t)elem_bytes};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(tm, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SVDQ_OK;
+}
+
+size_t scale_bytes(int64_t rows, int64_t K) { return (size_t)((rows + 127) / 128) * (size_t)(K / 64) * 512u; }
+
+// ---------------------------------------------------------------- launchers
+template <int RANK, bool QUANT>
+svdq_status launch_quant_t(const svdq_shape& s, const void* X, const float* inv, const void* L1p, void* Qx, void* Sx,
+                           void* T, cudaStream_t st) {
+  const int rows = QUANT ? (int)((s.M + 127) / 128 * 128) : (int)((s.M + 15) / 16 * 16);
+  const int grid = rows / svdq::kQuantRows;
+  const size_t smem = RANK > 0 ? (size_t)8 * svdq::kQuantRows * RANK * sizeof(float) : 0;
+  auto kern = svdq::quantize_act_kernel<RANK, QUANT>;
+  if (smem > 48 * 1024) SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  kern<<<grid, svdq::kQuantThreads, smem, st>>>(
+      static_cast<const __nv_bfloat16*>(X), inv, static_cast<const __nv_bfloat16*>(L1p), static_cast<uint8_t*>(Qx),
+      static_cast<uint8_t*>(Sx), static_cast<__nv_bfloat16*>(T), (int)s.M, (int)s.K);
+  SVDQ_LAUNCHED("quantize_act_kernel");
+  return SVDQ_OK;
+}
+
+template <bool QUANT>
+svdq_status launch_quant(const svdq_shape& s, int rank, const void* X, const float* inv, const void* L1p, void* Qx,
+                         void* Sx, void* T, cudaStream_t st) {
+  switch (rank) {
+#define SVDQ_CASE(R) \
+  case R:            \
+    return launch_quant_t<R, QUANT>(s, X, inv, L1p, Qx, Sx, T, st);
+    SVDQ_CASE(0) SVDQ_CASE(16) SVDQ_CASE(32) SVDQ_CASE(48) SVDQ_CASE(64) SVDQ_CASE(80) SVDQ_CASE(96)
+    SVDQ_CASE(112) SVDQ_CASE(128)
+#undef SVDQ_CASE
+    default:
+      return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d", rank);
+  }
+}
+
+template <int STAGES, int RANK>
+svdq_status launch_gemm_t(const svdq_shape& s, const CUtensorMap& tqx, const CUtensorMap& tqr, const CUtensorMap& tt,
+                          const CUtensorMap& tl, const void* Sx, const void* Sr, void* Y, cudaStream_t st) {
+  using L = svdq::GemmSmem<STAGES, RANK>;
+  auto kern = svdq::svdq_gemm_kernel<STAGES, RANK>;
+  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  dim3 grid((unsigned)(s.N / svdq::kGemmBN), (unsigned)((s.M + svdq::kGemmBM - 1) / svdq::kGemmBM));
+  kern<<<grid, svdq::kGemmThreads, L::kBytes, st>>>(tqx, tqr, tt, tl, static_cast<const uint8_t*>(Sx),
+                                                    static_cast<const uint8_t*>(Sr), static_cast<__nv_bfloat16*>(Y),
+                                                    (int)s.M, (int)s.N, (int)s.K);
+  SVDQ_LAUNCHED("svdq_gemm_kernel");
+  return SVDQ_OK;
+}
+
+constexpr int kGemmStages = 4;
+
+svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                        const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+  CUtensorMap tqx, tqr, tt, tl;
+  svdq_status r;
+  if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.N, 128, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if (rank > 0) {
+    if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.M, 16, 128,
+                       CU_TENSOR_MAP_SWIZZLE_32B)) != SVDQ_OK)
+      return r;
+    if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.N, 16, 128,
+                       CU_TENSOR_MAP_SWIZZLE_32B)) != SVDQ_OK)
+      return r;
+  } else {
+    memset(&tt, 0, sizeof(tt));
+    memset(&tl, 0, sizeof(tl));
+  }
+  switch (rank) {
+#define SVDQ_CASE(R) \
+  case R:            \
+    return launch_gemm_t<kGemmStages, R>(s, tqx, tqr, tt, tl, Sx, Sr, Y, st);
+    SVDQ_CASE(0) SVDQ_CASE(16) SVDQ_CASE(32) SVDQ_CASE(48) SVDQ_CASE(64) SVDQ_CASE(80) SVDQ_CASE(96)
+    SVDQ_CASE(112) SVDQ_CASE(128)
+#undef SVDQ_CASE
+    default:
+      return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d", rank);
+  }
+}
+
+template <int RANK>
+svdq_status launch_up_rmw_t(const svdq_shape& s, const void* T, const void* L2t, void* Y, cudaStream_t st) {
+  constexpr int LDS = RANK + 8;
+  const size_t smem_in = (size_t)(64 + 128) * LDS * 2, smem_out = (size_t)64 * 128 * 4;
+  const size_t smem = smem_in > smem_out ? smem_in : smem_out;
+  auto kern = svdq::lowrank_up_rmw_kernel<RANK>;
+  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+  dim3 grid((unsigned)(s.N / 128), (unsigned)((s.M + 63) / 64));
+  kern<<<grid, 128, smem, st>>>(static_cast<const __nv_bfloat16*>(T), static_cast<const __nv_bfloat16*>(L2t),
+                                static_cast<__nv_bfloat16*>(Y), (int)s.M, (int)s.N);
+  SVDQ_LAUNCHED("lowrank_up_rmw_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status launch_up_rmw(const svdq_shape& s, int rank, const void* T, const void* L2t, void* Y, cudaStream_t st) {
+  switch (rank) {
+#define SVDQ_CASE(R) \
+  case R:            \
+    return launch_up_rmw_t<R>(s, T, L2t, Y, st);
+    SVDQ_CASE(16) SVDQ_CASE(32) SVDQ_CASE(48) SVDQ_CASE(64) SVDQ_CASE(80) SVDQ_CASE(96) SVDQ_CASE(112)
+    SVDQ_CASE(128)
+#undef SVDQ_CASE
+    default:
+      return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d", rank);
+  }
+}
+
+svdq_status launch_channel_amax(int64_t rows, int64_t K, const void* X, float* amax, cudaStream_t st) {
+  SVDQ_CUDA(cudaMemsetAsync(amax, 0, (size_t)K * sizeof(float), st));
+  if (rows == 0) return SVDQ_OK;
+  const int threads = 128;
+  const int cols8 = (int)(K / 8);
+  const int gx = (cols8 + threads - 1) / threads;
+  // enough row blocks to fill the GPU several times over, each >= 32 rows
+  int gy = (int)((rows + 31) / 32);
+  const int max_gy = (4 * 148 + gx - 1) / gx;
+  if (gy > max_gy) gy = max_gy;
+  if (gy < 1) gy = 1;
+  const int rows_per_block = (int)((rows + gy - 1) / gy);
+  gy = (int)((rows + rows_per_block - 1) / rows_per_block);
+  svdq::channel_amax_kernel<<<dim3(gx, gy), threads, 0, st>>>(static_cast<const __nv_bfloat16*>(X), amax, (int)rows,
+                                                             (int)K, rows_per_block);
+  SVDQ_LAUNCHED("channel_amax_kernel");
+  return SVDQ_OK;
+}
+
+}  // namespace
+
+// ============================================================================ C ABI
+extern "C" {
+
+const char* svdq_status_string(int status) {
+  switch (status) {
+    case SVDQ_OK: return "SVDQ_OK";
+    case SVDQ_ERR_INVALID_ARG: return "SVDQ_ERR_INVALID_ARG";
+    case SVDQ_ERR_UNSUPPORTED_SHAPE: return "SVDQ_ERR_UNSUPPORTED_SHAPE";
+    case SVDQ_ERR_MISALIGNED: return "SVDQ_ERR_MISALIGNED";
+    case SVDQ_ERR_BUFFER_TOO_SMALL: return "SVDQ_ERR_BUFFER_TOO_SMALL";
+    case SVDQ_ERR_NO_DEVICE: return "SVDQ_ERR_NO_DEVICE";
+    case SVDQ_ERR_CUDA: return "SVDQ_ERR_CUDA";
+    case SVDQ_ERR_TIMEOUT: return "SVDQ_ERR_TIMEOUT";
+    case SVDQ_ERR_INTERNAL: return "SVDQ_ERR_INTERNAL";
+    default: return "SVDQ_ERR_UNKNOWN";
+  }
+}
+
+const char* svdq_last_error(void) { return g_last_error; }
+
+int svdq_version(void) { return 100; }
+
+svdq_status svdq_act_sizes(svdq_shape s, size_t* qx, size_t* sx, size_t* t) {
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (qx) *qx = (size_t)s.M * (size_t)(s.K / 2);
+  if (sx) *sx = scale_bytes(s.M, s.K);
+  if (t) *t = (size_t)s.M * (size_t)s.rank * 2u;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_weight_sizes(svdq_shape s, size_t* qr, size_t* sr, size_t* l1p, size_t* l2t, size_t* ws) {
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (qr) *qr = (size_t)s.N * (size_t)(s.K / 2);
+  if (sr) *sr = scale_bytes(s.N, s.K);
+  if (l1p) *l1p = (size_t)s.rank * (size_t)s.K * 2u;
+  if (l2t) *l2t = (size_t)s.N * (size_t)s.rank * 2u;
+  if (ws) *ws = svdq::svd_workspace_bytes(s.K, s.N, s.rank);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_channel_amax(int64_t M, int64_t K, const void* X, float* amax, void* stream) {
+  g_last_error[0] = 0;
+  if (M < 1 || K < 8 || K % 8 || K > (1ll << 30)) return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "amax shape M=%lld K=%lld", (long long)M, (long long)K);
+  if (!X || !amax) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(X) || !aligned16(amax)) return fail(SVDQ_ERR_MISALIGNED, "X and amax must be 16-byte aligned");
+  svdq_status r = check_device();
+  if (r != SVDQ_OK) return r;
+  return launch_channel_amax(M, K, X, amax, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_prepare_weights(svdq_shape s, const void* W, const float* act_amax, float alpha, unsigned int flags,
+                                 void* L1p, void* L2t, void* Qr, void* Sr, float* lambda, float* inv_lambda,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (!(alpha >= 0.f && alpha <= 1.f)) return fail(SVDQ_ERR_INVALID_ARG, "alpha must be in [0, 1]");
+  if (flags & ~(unsigned)SVDQ_PREPARE_GIVEN_FACTORS) return fail(SVDQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  if (!W || !act_amax || !Qr || !Sr || !lambda || !inv_lambda || (s.rank > 0 && (!L1p || !L2t)))
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {W, act_amax, Qr, Sr, lambda, inv_lambda, L1p, L2t, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  const bool given = (flags & SVDQ_PREPARE_GIVEN_FACTORS) != 0;
+  const size_t need = given ? 0 : svdq::svd_workspace_bytes(s.K, s.N, s.rank);
+  if (workspace_bytes < need || (need > 0 && !workspace))
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "workspace of %zu bytes needed", need);
+  if ((r = check_device()) != SVDQ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // weight channel maxima into the lambda buffer, then lambda / inv_lambda
+  if ((r = launch_channel_amax(s.N, s.K, W, inv_lambda, st)) != SVDQ_OK) return r;
+  svdq::smoothing_lambda_kernel<<<(unsigned)((s.K + 255) / 256), 256, 0, st>>>(act_amax, inv_lambda, alpha, lambda,
+                                                                              inv_lambda, (int)s.K);
+  SVDQ_LAUNCHED("smoothing_lambda_kernel");
+  if (s.rank > 0 && !given) {
+    if ((r = svdq::svd_lowrank_factors(s.K, s.N, s.rank, static_cast<const __nv_bfloat16*>(W), lambda,
+                                       static_cast<__nv_bfloat16*>(L1p), static_cast<__nv_bfloat16*>(L2t), workspace,
+                                       st, &set_error)) != SVDQ_OK)
+      return r;
+  }
+  const long long n_threads = s.N * (s.K / 16);
+  svdq::residual_quantize_kernel<<<(unsigned)((n_threads + 127) / 128), 128, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(W), lambda, static_cast<const __nv_bfloat16*>(L1p),
+      static_cast<const __nv_bfloat16*>(L2t), static_cast<uint8_t*>(Qr), static_cast<uint8_t*>(Sr), (int)s.N,
+      (int)s.K, (int)s.rank);
+  SVDQ_LAUNCHED("residual_quantize_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_act(svdq_shape s, const void* X, const float* inv_lambda, const void* L1p, void* Qx,
+                              void* Sx, void* T, int variant, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (variant != SVDQ_FUSED && variant != SVDQ_UNFUSED) return fail(SVDQ_ERR_INVALID_ARG, "variant %d", variant);
+  if (s.M == 0) return SVDQ_OK;
+  if (!X || !inv_lambda || !Qx || !Sx || (s.rank > 0 && (!L1p || !T))) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {X, inv_lambda, Qx, Sx, L1p, T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (variant == SVDQ_FUSED) return launch_quant<true>(s, s.rank, X, inv_lambda, L1p, Qx, Sx, T, st);
+  if ((r = launch_quant<true>(s, 0, X, inv_lambda, nullptr, Qx, Sx, nullptr, st)) != SVDQ_OK) return r;
+  if (s.rank == 0) return SVDQ_OK;
+  return launch_quant<false>(s, s.rank, X, nullptr, L1p, nullptr, nullptr, T, st);
+}
+
+svdq_status svdq_linear(svdq_shape s, const void* Qx, const void* Sx, const void* T, const void* Qr, const void* Sr,
+                        const void* L2t, void* Y, int variant, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (variant != SVDQ_FUSED && variant != SVDQ_UNFUSED) return fail(SVDQ_ERR_INVALID_ARG, "variant %d", variant);
+  if (s.M == 0) return SVDQ_OK;
+  if (!Qx || !Sx || !Qr || !Sr || !Y || (s.rank > 0 && (!T || !L2t))) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {Qx, Sx, T, Qr, Sr, L2t, Y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (variant == SVDQ_FUSED) return launch_gemm(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
+  if ((r = launch_gemm(s, 0, Qx, Sx, nullptr, Qr, Sr, nullptr, Y, st)) != SVDQ_OK) return r;
+  if (s.rank == 0) return SVDQ_OK;
+  return launch_up_rmw(s, s.rank, T, L2t, Y, st);
+}
+
+svdq_status svdq_scales_to_canonical(int64_t rows, int64_t K, const void* native, void* canonical, void* stream) {
+  g_last_error[0] = 0;
+  if (rows < 0 || K < 64 || K % 64 || K > (1ll << 20) || rows > (1ll << 31) - 1)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rows=%lld K=%lld", (long long)rows, (long long)K);
+  if (rows == 0) return SVDQ_OK;
+  if (!native || !canonical) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  svdq_status r = check_device();
+  if (r != SVDQ_OK) return r;
+  const size_t n = (size_t)rows * (size_t)(K / 16);
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  svdq::scales_native_to_canonical_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(native), static_cast<uint8_t*>(canonical), (int)rows, (int)K);
+  SVDQ_LAUNCHED("scales_native_to_canonical_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_check(void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_device();
+  if (r != SVDQ_OK) return r;
+  SVDQ_CUDA(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  SVDQ_CUDA(cudaGetLastError());
+  unsigned int word = 0, zero = 0;
+  SVDQ_CUDA(cudaMemcpyFromSymbol(&word, svdq::g_device_error, sizeof(word)));
+  if (word != 0) {
+    SVDQ_CUDA(cudaMemcpyToSymbol(svdq::g_device_error, &zero, sizeof(zero)));
+    return fail(SVDQ_ERR_TIMEOUT, "a kernel gave up on a bounded wait (device error %u)", word);
+  }
+  return SVDQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,304 @@
+// Activation-side kernels of the SVDQuant W4A4 layer:
+//   * quantize_act_kernel: smoothing, NVFP4 group quantization and (fused)
+//     the low-rank down-projection T = X L1' from one read of X
+//     (devpress.csdn.net SVDQuant walkthrough, eq. (1), eq. (5), Fig. 6);
+//   * channel_amax_kernel: per-channel max|x| (handbook SmoothQuant section);
+//   * scales_native_to_canonical_kernel: inspection helper.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
+#include "svdq_ptx.cuh"
+
+namespace svdq {
+
+// Byte offset of scale (row r, 16-group g) in the native tile layout
+// (128-row x 64-element atoms of 512 bytes; see include/svdq.h).
+__host__ __device__ __forceinline__ size_t native_scale_offset(int r, int g, int K) {
+  const int kb = g >> 2, j = g & 3;
+  const int rb = r >> 7, rr = r & 127;
+  return ((size_t)rb * (size_t)(K >> 6) + (size_t)kb) * 512u + 16u * (rr & 31) + 4u * (rr >> 5) + j;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// NVFP4 encoding of 16 fp32 values (one group):
+//   s = E4M3_rne_satfinite(fp32(max|v| / 6)); q_i = E2M1_rne_satfinite(fp32(v_i * fp32(1/s)));
+//   all codes +0 when s decodes to 0. Element 2i lands in the low nibble of byte i.
+__device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& codes, uint32_t& sbyte) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  const float s32 = __fdiv_rn(amax, 6.0f);
+  const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(s32, __NV_SATFINITE, __NV_E4M3);
+  const float sval = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
+  sbyte = (uint32_t)sb;
+  if (sval == 0.f) {
+    codes = make_uint2(0u, 0u);
+    return;
+  }
+  const float inv = __frcp_rn(sval);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int b = 0; b < 8; ++b) {
+    const float2 p = make_float2(__fmul_rn(v[2 * b], inv), __fmul_rn(v[2 * b + 1], inv));
+    const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(p, __NV_E2M1, cudaRoundNearest);
+    w[b >> 2] |= (byte & 0xFFu) << (8 * (b & 3));
+  }
+  codes = make_uint2(w[0], w[1]);
+}
+
+// One 16-element chunk of a bf16 row: 2 x 16-byte loads.
+struct Chunk16 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ Chunk16 load_chunk16(const __nv_bfloat16* p, bool ok) {
+  Chunk16 c;
+  if (ok) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+    c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
+    c.w[4] = b.x; c.w[5] = b.y; c.w[6] = b.z; c.w[7] = b.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) c.w[i] = 0u;
+  }
+  return c;
+}
+
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+constexpr int kQuantThreads = 256;   // 8 warps
+constexpr int kQuantRows = 16;       // rows per CTA (one m16 MMA tile)
+
+// Grid: one CTA per 16 rows of ceil(M/128)*128 rows (padding rows only write
+// zero scales so the native scale atoms are fully defined). Warp w walks the
+// 64-column slabs w, w+8, ...; thread (g = lane/4, t = lane%4) owns rows
+// m0+g and m0+g+8, columns [64 s + 16 t, +16) of slab s — one quantization
+// group per row. The down-projection reuses the same registers as mma.sync
+// A fragments: in k-step ks of a slab, the MMA's reduction index
+// {2t, 2t+1, 2t+8, 2t+9} maps to columns 64 s + 16 t + 4 ks + {0, 1, 2, 3}, and
+// the B fragment (L1p row n, same columns) is one 8-byte piece of L1p.
+// Partial T of the 8 warps is summed in shared memory in fixed warp order.
+template <int RANK, bool QUANT>
+__global__ void __launch_bounds__(kQuantThreads) quantize_act_kernel(
+    const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
+    const __nv_bfloat16* __restrict__ L1p, uint8_t* __restrict__ Qx, uint8_t* __restrict__ Sx,
+    __nv_bfloat16* __restrict__ T, int M, int K) {
+  constexpr int NT = RANK / 8;
+  extern __shared__ float red[];   // [8][16][RANK]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int m0 = blockIdx.x * kQuantRows;
+  const int rA = m0 + g, rB = m0 + g + 8;
+  const bool okA = rA < M, okB = rB < M;
+  const int nslab = K >> 6;
+  const size_t ldq = (size_t)K >> 1;
+
+  float acc[NT > 0 ? NT : 1][4];
+#pragma unroll
+  for (int i = 0; i < (NT > 0 ? NT : 1); ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+
+  if (m0 < M || QUANT) {
+#pragma unroll 1
+    for (int s = warp; s < nslab; s += 8) {
+      const int c = s * 64 + t * 16;
+      const Chunk16 xa = load_chunk16(X + (size_t)rA * K + c, okA);
+      const Chunk16 xb = load_chunk16(X + (size_t)rB * K + c, okB);
+
+      if constexpr (QUANT) {
+        float il[16];
+        const float4* ilp = reinterpret_cast<const float4*>(inv_lambda + c);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float4 f = __ldg(ilp + q);
+          il[4 * q] = f.x; il[4 * q + 1] = f.y; il[4 * q + 2] = f.z; il[4 * q + 3] = f.w;
+        }
+        uint32_t sbA, sbB;
+        uint2 qa, qb;
+        {
+          float v[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __fmul_rn(bf16lo(xa.w[i]), il[2 * i]);
+            v[2 * i + 1] = __fmul_rn(bf16hi(xa.w[i]), il[2 * i + 1]);
+          }
+          nvfp4_encode16(v, qa, sbA);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            v[2 * i] = __fmul_rn(bf16lo(xb.w[i]), il[2 * i]);
+            v[2 * i + 1] = __fmul_rn(bf16hi(xb.w[i]), il[2 * i + 1]);
+          }
+          nvfp4_encode16(v, qb, sbB);
+        }
+        if (okA) *reinterpret_cast<uint2*>(Qx + (size_t)rA * ldq + (c >> 1)) = qa;
+        if (okB) *reinterpret_cast<uint2*>(Qx + (size_t)rB * ldq + (c >> 1)) = qb;
+        // The four scale bytes of one row and slab are adjacent in the native
+        // layout (group j = t): gather them to lane t == 0 and store one word.
+        const uint32_t a1 = __shfl_down_sync(0xFFFFFFFFu, sbA, 1), a2 = __shfl_down_sync(0xFFFFFFFFu, sbA, 2),
+                       a3 = __shfl_down_sync(0xFFFFFFFFu, sbA, 3);
+        const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sbB, 1), b2 = __shfl_down_sync(0xFFFFFFFFu, sbB, 2),
+                       b3 = __shfl_down_sync(0xFFFFFFFFu, sbB, 3);
+        if (t == 0) {
+          *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rA, s * 4, K)) =
+              sbA | (a1 << 8) | (a2 << 16) | (a3 << 24);
+          *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rB, s * 4, K)) =
+              sbB | (b1 << 8) | (b2 << 16) | (b3 << 24);
+        }
+      }
+
+      if constexpr (NT > 0) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const Chunk16 l = load_chunk16(L1p + (size_t)(nt * 8 + g) * K + c, true);
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16_16816(acc[nt], xa.w[2 * ks], xb.w[2 * ks], xa.w[2 * ks + 1], xb.w[2 * ks + 1],
+                           l.w[2 * ks], l.w[2 * ks + 1]);
+        }
+      }
+    }
+  }
+
+  if constexpr (NT > 0) {
+    float* mine = red + (size_t)warp * kQuantRows * RANK;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int col = nt * 8 + 2 * t;
+      mine[g * RANK + col] = acc[nt][0];
+      mine[g * RANK + col + 1] = acc[nt][1];
+      mine[(g + 8) * RANK + col] = acc[nt][2];
+      mine[(g + 8) * RANK + col + 1] = acc[nt][3];
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < kQuantRows * RANK; e += kQuantThreads) {
+      float s = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) s += red[w * kQuantRows * RANK + e];
+      const int row = m0 + e / RANK;
+      if (row < M) T[(size_t)row * RANK + (e % RANK)] = __float2bfloat16_rn(s);
+    }
+  }
+}
+
+// amax[j] = max_m |X[m][j]| over bf16 X [M][K]; amax must be zeroed first.
+// Each thread owns 8 adjacent columns and a strided set of rows; non-negative
+// floats order like their bit patterns, so an integer atomicMax is exact.
+__global__ void channel_amax_kernel(const __nv_bfloat16* __restrict__ X, float* __restrict__ amax, int M, int K,
+                                    int rows_per_block) {
+  const int col8 = (blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (col8 >= K) return;
+  const int r0 = blockIdx.y * rows_per_block;
+  const int r1 = min(M, r0 + rows_per_block);
+  float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int r = r0; r < r1; ++r) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + (size_t)r * K + col8));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      m[2 * i] = fmaxf(m[2 * i], fabsf(bf16lo(w[i])));
+      m[2 * i + 1] = fmaxf(m[2 * i + 1], fabsf(bf16hi(w[i])));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    atomicMax(reinterpret_cast<unsigned int*>(amax) + col8 + i, __float_as_uint(m[i]));
+}
+
+__global__ void scales_native_to_canonical_kernel(const uint8_t* __restrict__ native, uint8_t* __restrict__ canon,
+                                                  int rows, int K) {
+  const int G = K >> 4;
+  const size_t n = (size_t)rows * G;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i / G), g = (int)(i % G);
+    canon[i] = native[native_scale_offset(r, g, K)];
+  }
+}
+
+// Unfused up-projection: Y = bf16(fp32(Y) + T L2t^T). A CTA (4 warps) owns a
+// 64 x 128 tile of Y; T and L2t tiles are staged in shared memory, each warp
+// computes 16 rows x 128 columns with mma.sync, the fp32 results go through
+// shared memory so that Y is read and written with coalesced 16-byte accesses.
+template <int RANK>
+__global__ void __launch_bounds__(128) lowrank_up_rmw_kernel(const __nv_bfloat16* __restrict__ T,
+                                                             const __nv_bfloat16* __restrict__ L2t,
+                                                             __nv_bfloat16* __restrict__ Y, int M, int N) {
+  constexpr int BM = 64, BN = 128, LDS = RANK + 8;   // +8 bf16 pads rows against bank conflicts
+  extern __shared__ __align__(16) unsigned char up_smem[];
+  __nv_bfloat16* Ts = reinterpret_cast<__nv_bfloat16*>(up_smem);
+  __nv_bfloat16* Ls = Ts + BM * LDS;
+  float* Ys = reinterpret_cast<float*>(up_smem);      // reused after the MMAs: [BM][BN]
+  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+
+  for (int i = threadIdx.x; i < BM * RANK / 8; i += 128) {
+    const int r = i / (RANK / 8), c = (i % (RANK / 8)) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (m0 + r < M) v = __ldg(reinterpret_cast<const uint4*>(T + (size_t)(m0 + r) * RANK + c));
+    *reinterpret_cast<uint4*>(Ts + r * LDS + c) = v;
+  }
+  for (int i = threadIdx.x; i < BN * RANK / 8; i += 128) {
+    const int r = i / (RANK / 8), c = (i % (RANK / 8)) * 8;
+    *reinterpret_cast<uint4*>(Ls + r * LDS + c) =
+        __ldg(reinterpret_cast<const uint4*>(L2t + (size_t)(n0 + r) * RANK + c));
+  }
+  __syncthreads();
+
+  float acc[BN / 8][4];
+#pragma unroll
+  for (int i = 0; i < BN / 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+  const __nv_bfloat16* Tw = Ts + warp * 16 * LDS;
+#pragma unroll
+  for (int ks = 0; ks < RANK / 16; ++ks) {
+    const int k = ks * 16 + 2 * t;
+    const uint32_t a0 = *reinterpret_cast<const uint32_t*>(Tw + g * LDS + k);
+    const uint32_t a1 = *reinterpret_cast<const uint32_t*>(Tw + (g + 8) * LDS + k);
+    const uint32_t a2 = *reinterpret_cast<const uint32_t*>(Tw + g * LDS + k + 8);
+    const uint32_t a3 = *reinterpret_cast<const uint32_t*>(Tw + (g + 8) * LDS + k + 8);
+#pragma unroll
+    for (int nt = 0; nt < BN / 8; ++nt) {
+      const __nv_bfloat16* Lr = Ls + (nt * 8 + g) * LDS + k;
+      mma_bf16_16816(acc[nt], a0, a1, a2, a3, *reinterpret_cast<const uint32_t*>(Lr),
+                     *reinterpret_cast<const uint32_t*>(Lr + 8));
+    }
+  }
+  __syncthreads();   // Ts/Ls no longer needed: reuse the space for the fp32 tile
+#pragma unroll
+  for (int nt = 0; nt < BN / 8; ++nt) {
+    const int col = nt * 8 + 2 * t, row = warp * 16 + g;
+    Ys[row * BN + col] = acc[nt][0];
+    Ys[row * BN + col + 1] = acc[nt][1];
+    Ys[(row + 8) * BN + col] = acc[nt][2];
+    Ys[(row + 8) * BN + col + 1] = acc[nt][3];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < BM * BN / 8; i += 128) {
+    const int r = i / (BN / 8), c = (i % (BN / 8)) * 8;
+    if (m0 + r >= M) continue;
+    uint4* yp = reinterpret_cast<uint4*>(Y + (size_t)(m0 + r) * N + n0 + c);
+    const uint4 y = *yp;
+    const uint32_t w[4] = {y.x, y.y, y.z, y.w};
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float lo = bf16lo(w[q]) + Ys[r * BN + c + 2 * q];
+      const float hi = bf16hi(w[q]) + Ys[r * BN + c + 2 * q + 1];
+      const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+      o[q] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+    *yp = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+}  // namespace svdq

@@ -1,0 +1,200 @@
+"""Python binding of the SVDQuant W4A4 C ABI (include/svdq.h).
+
+Argument marshalling only: every step of the layer runs in the CUDA library
+``libsvdq.so`` built in this directory. Tensors are torch CUDA tensors; calls
+are issued on torch's current CUDA stream. There is no CPU fallback: if the
+library is missing or the device is not sm_100, calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+SVDQ_FUSED = 0
+SVDQ_UNFUSED = 1
+SVDQ_PREPARE_GIVEN_FACTORS = 1
+
+STATUS = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_SHAPE", 3: "SVDQ_ERR_MISALIGNED",
+    4: "SVDQ_ERR_BUFFER_TOO_SMALL", 5: "SVDQ_ERR_NO_DEVICE", 6: "SVDQ_ERR_CUDA", 7: "SVDQ_ERR_TIMEOUT",
+    8: "SVDQ_ERR_INTERNAL",
+}
+
+# Every symbol the header declares, with its ctypes signature.
+EXPORTS = [
+    "svdq_status_string", "svdq_last_error", "svdq_version", "svdq_act_sizes", "svdq_weight_sizes",
+    "svdq_channel_amax", "svdq_prepare_weights", "svdq_quantize_act", "svdq_linear",
+    "svdq_scales_to_canonical", "svdq_check",
+]
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("M", ctypes.c_int64), ("K", ctypes.c_int64), ("N", ctypes.c_int64), ("rank", ctypes.c_int32)]
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m w4a4_diffusion_model_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, sz, i64, st = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int64, ctypes.c_int
+    P = ctypes.POINTER
+    lib.svdq_status_string.argtypes, lib.svdq_status_string.restype = [ctypes.c_int], ctypes.c_char_p
+    lib.svdq_last_error.argtypes, lib.svdq_last_error.restype = [], ctypes.c_char_p
+    lib.svdq_version.argtypes, lib.svdq_version.restype = [], ctypes.c_int
+    lib.svdq_act_sizes.argtypes, lib.svdq_act_sizes.restype = [Shape, P(sz), P(sz), P(sz)], st
+    lib.svdq_weight_sizes.argtypes = [Shape, P(sz), P(sz), P(sz), P(sz), P(sz)]
+    lib.svdq_weight_sizes.restype = st
+    lib.svdq_channel_amax.argtypes, lib.svdq_channel_amax.restype = [i64, i64, vp, vp, vp], st
+    lib.svdq_prepare_weights.argtypes = [Shape, vp, vp, ctypes.c_float, ctypes.c_uint, vp, vp, vp, vp, vp, vp,
+                                         vp, sz, vp]
+    lib.svdq_prepare_weights.restype = st
+    lib.svdq_quantize_act.argtypes = [Shape, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
+    lib.svdq_quantize_act.restype = st
+    lib.svdq_linear.argtypes = [Shape, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
+    lib.svdq_linear.restype = st
+    lib.svdq_scales_to_canonical.argtypes, lib.svdq_scales_to_canonical.restype = [i64, i64, vp, vp, vp], st
+    lib.svdq_check.argtypes, lib.svdq_check.restype = [vp], st
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise SvdqError(status, load().svdq_last_error().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+@dataclass(frozen=True)
+class LayerShape:
+    M: int
+    K: int
+    N: int
+    rank: int
+
+    def c(self) -> Shape:
+        return Shape(self.M, self.K, self.N, self.rank)
+
+
+def svdq_act_sizes(shape: LayerShape) -> tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().svdq_act_sizes(shape.c(), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def svdq_weight_sizes(shape: LayerShape) -> tuple[int, int, int, int, int]:
+    v = [ctypes.c_size_t() for _ in range(5)]
+    _check(load().svdq_weight_sizes(shape.c(), *[ctypes.byref(x) for x in v]))
+    return tuple(x.value for x in v)
+
+
+def svdq_channel_amax(X: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    M, K = X.shape
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=X.device)
+    _check(load().svdq_channel_amax(M, K, _ptr(X), _ptr(out), _stream()))
+    return out
+
+
+@dataclass
+class PreparedWeights:
+    shape: LayerShape          # M is unused (0)
+    Qr: torch.Tensor
+    Sr: torch.Tensor
+    L1p: torch.Tensor | None
+    L2t: torch.Tensor | None
+    lam: torch.Tensor
+    inv_lam: torch.Tensor
+
+
+def svdq_prepare_weights(W_lin: torch.Tensor, act_amax: torch.Tensor, alpha: float, rank: int,
+                         L1p: torch.Tensor | None = None, L2t: torch.Tensor | None = None) -> PreparedWeights:
+    """Smoothing, top-rank split and residual NVFP4 encoding of W_lin [N][K].
+    Pass both L1p [rank][K] and L2t [N][rank] (bf16) to use given factors."""
+    N, K = W_lin.shape
+    shape = LayerShape(0, K, N, rank)
+    qr, sr, l1, l2, ws = svdq_weight_sizes(shape)
+    dev = W_lin.device
+    given = L1p is not None and L2t is not None
+    if not given:
+        L1p = torch.empty(rank, K, dtype=torch.bfloat16, device=dev) if rank else None
+        L2t = torch.empty(N, rank, dtype=torch.bfloat16, device=dev) if rank else None
+    Qr = torch.empty(qr, dtype=torch.uint8, device=dev)
+    Sr = torch.empty(sr, dtype=torch.uint8, device=dev)
+    lam = torch.empty(K, dtype=torch.float32, device=dev)
+    inv = torch.empty(K, dtype=torch.float32, device=dev)
+    work = torch.empty(ws, dtype=torch.uint8, device=dev) if (ws and not given) else None
+    _check(load().svdq_prepare_weights(
+        shape.c(), _ptr(W_lin), _ptr(act_amax), ctypes.c_float(alpha),
+        SVDQ_PREPARE_GIVEN_FACTORS if given else 0, _ptr(L1p), _ptr(L2t), _ptr(Qr), _ptr(Sr), _ptr(lam), _ptr(inv),
+        _ptr(work), ws if work is not None else 0, _stream()))
+    return PreparedWeights(shape, Qr.view(N, K // 2), Sr, L1p, L2t, lam, inv)
+
+
+def svdq_quantize_act(X: torch.Tensor, inv_lambda: torch.Tensor, L1p: torch.Tensor | None, rank: int, N: int = 128,
+                      variant: int = SVDQ_FUSED, out: tuple | None = None):
+    """Returns (Qx [M][K/2] uint8, Sx native uint8, T [M][rank] bf16 or None)."""
+    M, K = X.shape
+    shape = LayerShape(M, K, N, rank)
+    if out is None:
+        qx, sx, _ = svdq_act_sizes(shape)
+        Qx = torch.empty(M, K // 2, dtype=torch.uint8, device=X.device)
+        Sx = torch.empty(sx, dtype=torch.uint8, device=X.device)
+        T = torch.empty(M, rank, dtype=torch.bfloat16, device=X.device) if rank else None
+    else:
+        Qx, Sx, T = out
+    _check(load().svdq_quantize_act(shape.c(), _ptr(X), _ptr(inv_lambda), _ptr(L1p), _ptr(Qx), _ptr(Sx), _ptr(T),
+                                    variant, _stream()))
+    return Qx, Sx, T
+
+
+def svdq_linear(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: PreparedWeights,
+                variant: int = SVDQ_FUSED, out: torch.Tensor | None = None) -> torch.Tensor:
+    M = Qx.shape[0]
+    K, N, rank = W.shape.K, W.shape.N, W.shape.rank
+    shape = LayerShape(M, K, N, rank)
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Qx.device)
+    _check(load().svdq_linear(shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t), _ptr(Y),
+                              variant, _stream()))
+    return Y
+
+
+def svdq_scales_to_canonical(native: torch.Tensor, rows: int, K: int) -> torch.Tensor:
+    out = torch.empty(rows, K // 16, dtype=torch.uint8, device=native.device)
+    _check(load().svdq_scales_to_canonical(rows, K, _ptr(native), _ptr(out), _stream()))
+    return out
+
+
+def svdq_check() -> None:
+    _check(load().svdq_check(_stream()))
