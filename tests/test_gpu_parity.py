@@ -87,13 +87,15 @@ def test_codec_ties_saturation_and_signed_zero():
             row[16 * g:16 * g + 16] = grp
         rows.append(row)
     X = np.array(rows)
+    assert np.array_equal(O.bf16(X), X)            # the tie rows are exact in bf16
     X[5] = 0.0
     X[6, :16] = -0.0
-    X[7] = rng.standard_normal(K) * 1e-4           # scales underflow / subnormal
-    X[8] = rng.standard_normal(K) * 1e4            # E4M3 scale saturates at 448
+    X[7] = O.bf16(rng.standard_normal(K) * 1e-4)   # scales underflow / subnormal
+    X[8] = O.bf16(rng.standard_normal(K) * 1e4)    # E4M3 scale saturates at 448
     X[9, ::2] = -1e-30
+    X[9] = O.bf16(X[9])
     Xt = torch.from_numpy(X).to(torch.float32).to(torch.bfloat16)
-    assert np.array_equal(np64(Xt), X)             # every value is exact in bf16
+    assert np.array_equal(np64(Xt), X)
     inv = np.ones(K, dtype=np.float32)
     codes, scales, _ = O.quantize_act(np64(Xt), inv, np.zeros((K, 0)))
     Qx, Sx, _ = S.svdq_quantize_act(Xt.cuda(), torch.from_numpy(inv).cuda(), None, 0, 128)
