@@ -1,0 +1,488 @@
+"""Benchmark of the SVDQuant W4A4 linear layer on B200.
+
+One step = one pass of the per-call path over one batch of tokens:
+svdq_quantize_act (smoothing + NVFP4 quantization + fused low-rank
+down-projection) then svdq_linear (tcgen05 FP4 GEMM + fused up-projection),
+with X already resident in device memory. Metric: effective TFLOPS,
+FLOPs = 2MNK + 2Mr(K+N) per step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...      # the CPU oracle, timed on host cores
+
+Multi-GPU (launched by torchrun, one rank per GPU): every rank runs the layer
+on its own batch of tokens with the same weights (token rows are independent:
+no data-path collective); the step time is the max over ranks, the value the
+FLOPs of all ranks over that time (weak scaling).
+
+Timing: W untimed warm-up steps; each timed step is bracketed by CUDA events
+on the launching stream, with a write of a 256 MiB buffer (larger than the
+126 MB L2) between steps so that every step starts with a cold L2.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from w4a4_diffusion_model_b200 import synth  # noqa: E402
+
+METRIC = "SVDQuant W4A4 linear effective TFLOPS (2MNK + 2Mr(K+N)) per layer call, FLUX shapes"
+DEFAULT_WORKLOAD = synth.FLUX_QKV.name
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_PER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput ratio on B200 (9 : 2.25 PFLOP/s)
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=50)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--no-extras", action="store_true", help="skip the cuBLAS / unfused / rank-0 / e2e / CPU legs")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    p.add_argument("--extra-json", default=None, help="append per-leg details to this JSONL file")
+    return p.parse_args()
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def quantize_bytes(w: synth.Workload) -> int:
+    """Algorithmic HBM bytes of one quantize launch: read X, inv_lambda, L1p;
+    write codes, scales (rows padded to 128) and T."""
+    Mp = (w.M + 127) // 128 * 128
+    return 2 * w.M * w.K + 4 * w.K + 2 * w.rank * w.K + w.M * w.K // 2 + Mp * w.K // 16 + 2 * w.M * w.rank
+
+
+def gemm_flops(w: synth.Workload) -> int:
+    """Algorithmic FLOPs of one GEMM launch: 2MNK (FP4) + 2MrN (fused up-projection)."""
+    return 2 * w.M * w.N * w.K + 2 * w.M * w.rank * w.N
+
+
+def kernel_source_hash() -> str:
+    p = os.path.join(ROOT, "w4a4_diffusion_model_b200", "csrc", "svdq_gemm.cuh")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def profiled_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current kernel source for this workload; else None."""
+    p = os.path.join(ROOT, "profiles", f"svdq_gemm_{workload}.md")
+    if not os.path.exists(p):
+        return None
+    src_hash = kernel_source_hash()
+    with open(p) as f:
+        for line in f:
+            if line.startswith("traffic_bytes_per_launch:"):
+                parts = line.split()
+                if len(parts) >= 3 and parts[2] == src_hash:
+                    return float(parts[1])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while active.
+    summary(t0, t1) keeps the samples taken inside the host-time window
+    [t0, t1] (the timed region); if that window is shorter than the sampling
+    period it falls back to every sample taken while the GPU was loaded."""
+
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.out.close()
+
+    def n_samples(self) -> int:
+        try:
+            with open(self.path) as f:
+                return sum(1 for _ in f)
+        except Exception:
+            return 0
+
+    def summary(self, t0: float, t1: float, t_load: float):
+        if self.proc is None or not self.path:
+            return None
+        import datetime
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[6:10]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        window = "timed region"
+        if len(inside) < 2:
+            inside = [r for r in rows if t_load <= r[0] <= t1]
+            window = "spin-up + timed region (timed region shorter than the 200 ms sampling period)"
+        if not inside:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, _, flags in inside for i, fl in enumerate(flags) if fl == "Active"})
+        return {"sm_mhz": statistics.median(r[1] for r in inside), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+def smi_index(local: int) -> str:
+    """nvidia-smi --id of the GPU behind CUDA device `local`."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local < len(ids):
+            return ids[local]
+    return str(local)
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+def oracle_sample(w: synth.Workload, X_cpu: torch.Tensor, W_cpu: torch.Tensor, rows=64, cols=512):
+    """Set up the oracle's per-call path on a bounded sample: `rows` token rows
+    and `cols` output channels of the layer, full K. Returns (fn, flops)."""
+    import oracle as O  # only the CPU-baseline / reference legs use the oracle
+
+    rng = np.random.default_rng(w.seed + 17)
+    r_idx = np.sort(rng.choice(w.M, min(rows, w.M), replace=False))
+    c_idx = np.sort(rng.choice(w.N, min(cols, w.N), replace=False))
+    Xn = X_cpu.float().numpy().astype(np.float64)
+    Wn = W_cpu.float().numpy().astype(np.float64)
+    amax = O.channel_amax(Xn)
+    lam32, inv32 = O.smoothing_lambda(amax, Wn, w.alpha)
+    What_c = lam32.astype(np.float64)[:, None] * Wn[c_idx].T
+    U, S, Vt = np.linalg.svd(What_c, full_matrices=False)
+    L1p = O.bf16(U[:, :w.rank] * S[:w.rank] / lam32.astype(np.float64)[:, None])
+    L2 = O.bf16(Vt[:w.rank])
+    _, qr, sr = O.residual_quantize(Wn[c_idx], lam32, L1p, L2)
+    Xs = Xn[r_idx]
+
+    def fn():
+        qx, sx, T = O.quantize_act(Xs, inv32, L1p)
+        return O.linear(qx, sx, T, qr, sr, L2)
+
+    m, n = len(r_idx), len(c_idx)
+    flops = 2 * m * n * w.K + 2 * m * w.rank * (w.K + n)
+    sample = (f"oracle per-call path (quantize + down-projection + dequantized fp64 GEMM + up-projection) "
+              f"on {m} token rows x {n} output channels x K={w.K} of {w.name}; prepare excluded")
+    return fn, flops, sample
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_cpu(fn, flops, seconds):
+    fn()  # warm
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return flops * n / el / 1e12, n, el
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    X, W = synth.generate(w)
+    fn, flops, sample = oracle_sample(w, X, W)
+    for _ in range(args.warmup):
+        fn()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        fn()
+        times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = flops * len(times) / tot / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * tot / len(times), 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "M": w.M, "K": w.K, "N": w.N, "rank": w.rank, "sample": sample},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU leg
+def aggregate_max(value: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (identity at world size 1)."""
+    if world <= 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def lowrank_factors(W_dev: torch.Tensor, lam: torch.Tensor, rank: int):
+    """Top-rank split of W_hat = diag(lambda) W_lin^T (offline, untimed):
+    L1p [rank][K] = bf16(U_r S_r / lambda)^T, L2t [N][rank] = bf16(V_r)."""
+    What = (W_dev.double() * lam.double()[None, :]).T
+    U, S, Vh = torch.linalg.svd(What, full_matrices=False)
+    L1 = U[:, :rank] * S[:rank]
+    L1p = (L1 / lam.double()[:, None]).T.contiguous().float().to(torch.bfloat16)
+    L2t = Vh[:rank].T.contiguous().float().to(torch.bfloat16)
+    return L1p, L2t
+
+
+def run_ours(args):
+    from w4a4_diffusion_model_b200 import svdq as S
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank_id = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    S.load()
+
+    w = synth.WORKLOADS[args.workload]
+    X_cpu, W_cpu = synth.generate(w)
+    if rank_id > 0:          # each rank its own tokens, same weights
+        X_cpu, _ = synth.generate(w.with_(seed=w.seed + 7919 * rank_id))
+    X = X_cpu.to(dev)
+    W = W_cpu.to(dev)
+
+    # offline: calibration amax, smoothing, split, residual encoding (untimed)
+    amax = S.svdq_channel_amax(X)
+    P0 = S.svdq_prepare_weights(W, amax, w.alpha, 0)
+    factors = lowrank_factors(W, P0.lam, w.rank) if w.rank else (None, None)
+    P = S.svdq_prepare_weights(W, amax, w.alpha, w.rank, *factors)
+    torch.cuda.synchronize()
+
+    qx_b, sx_b, t_b = S.svdq_act_sizes(S.LayerShape(w.M, w.K, w.N, w.rank))
+    Qx = torch.empty(w.M, w.K // 2, dtype=torch.uint8, device=dev)
+    Sx = torch.empty(sx_b, dtype=torch.uint8, device=dev)
+    T = torch.empty(w.M, w.rank, dtype=torch.bfloat16, device=dev) if w.rank else None
+    Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(P_=P, variant=S.SVDQ_FUSED, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        S.svdq_quantize_act(X, P_.inv_lam, P_.L1p, P_.shape.rank, w.N, variant, out=(Qx, Sx, T if P_.shape.rank else None))
+        if ev is not None:
+            ev[1].record(stream)
+        S.svdq_linear(Qx, Sx, T if P_.shape.rank else None, P_, variant, out=Y)
+        if ev is not None:
+            ev[2].record(stream)
+
+    def timed(n, fn, warm=3):
+        for _ in range(warm):      # untimed: first-call setup (library handles, heuristics) stays out
+            flush.zero_()
+            fn([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        for i in range(n):
+            flush.zero_()
+            fn(evs[i])
+        torch.cuda.synchronize()
+        k1 = [evs[i][0].elapsed_time(evs[i][1]) for i in range(n)]
+        k2 = [evs[i][1].elapsed_time(evs[i][2]) for i in range(n)]
+        return k1, k2
+
+    with ClockSampler(smi_index(local)) as clk:
+        # spin-up: keep the GPU loaded until the sampler reports, then warm up
+        t_load = time.time()
+        t_end = t_load + 1.5
+        while time.time() < t_end and (clk.n_samples() < 2 or time.time() < t_load + 0.6):
+            for _ in range(20):
+                step()
+            torch.cuda.synchronize()
+        for _ in range(args.warmup):
+            step()
+        S.svdq_check()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t0 = time.time()
+        k1, k2 = timed(args.steps, lambda ev: step(ev=ev), warm=0)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        if world > 1:
+            torch.distributed.barrier()
+        time.sleep(0.25)
+    S.svdq_check()
+    clocks = clk.summary(t0 - 0.2, t1 + 0.2, t_load)
+
+    step_ms = [a + b for a, b in zip(k1, k2)]
+    total_ms = aggregate_max(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    flops_step = w.flops()
+    value = flops_step * world / (ms_per_step * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
+    k2_ms = statistics.mean(k2)
+    k1_ms = statistics.mean(k1)
+    achieved = gemm_flops(w) / (k2_ms * 1e-3) / 1e12
+    traffic = profiled_traffic(w.name)
+    roofline = {"bound": "tensor", "kernel": "svdq_gemm_kernel", "achieved": round(achieved, 2),
+                "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
+                "traffic": traffic,
+                "peak_note": f"dense FP4 = {FP4_PER_BF16:g} x {peak_src} sustained bf16 "
+                             f"{peaks['bf16_tflops_sustained']:.1f} TFLOP/s; "
+                             f"vs 9000 TFLOP/s datasheet: {achieved / 9000:.4f}; "
+                             f"vs {FP4_PER_BF16:g} x burst bf16: {achieved / (FP4_PER_BF16 * peaks['bf16_tflops']):.4f}"}
+    q_gbs = quantize_bytes(w) / (k1_ms * 1e-3) / 1e9
+    roofline_q = {"bound": "hbm", "kernel": "quantize_act_kernel", "achieved": round(q_gbs, 1),
+                  "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / peaks["hbm_gbs"], 4),
+                  "algorithmic_bytes": quantize_bytes(w)}
+
+    extras = {}
+    e2e = None
+    cpu = None
+    if not args.no_extras:
+        n_x = max(5, args.steps // 2)
+        # unfused variant (same arithmetic, separate passes)
+        k1u, k2u = timed(n_x, lambda ev: step(variant=S.SVDQ_UNFUSED, ev=ev))
+        # no low-rank branch (rank 0) on the same shape
+        if w.rank:
+            k1z, k2z = timed(n_x, lambda ev: step(P_=P0, ev=ev))
+        else:
+            k1z, k2z = k1, k2
+        # bf16 cuBLAS X W^T through torch
+        def cublas(ev):
+            ev[0].record(stream)
+            torch.nn.functional.linear(X, W)
+            ev[1].record(stream)
+            ev[2].record(stream)
+        kc, _ = timed(n_x, cublas)
+        lay = statistics.mean(step_ms)
+        extras = {
+            "quantize_ms": round(k1_ms, 4), "gemm_ms": round(k2_ms, 4), "layer_ms": round(lay, 4),
+            "unfused_layer_ms": round(statistics.mean(a + b for a, b in zip(k1u, k2u)), 4),
+            "rank0_layer_ms": round(statistics.mean(a + b for a, b in zip(k1z, k2z)), 4),
+            "rank0_gemm_ms": round(statistics.mean(k2z), 4),
+            "bf16_cublas_ms": round(statistics.mean(kc), 4),
+            "bf16_cublas_tflops": round(2 * w.M * w.N * w.K / (statistics.mean(kc) * 1e-3) / 1e12, 1),
+        }
+        extras["lowrank_overhead_layer"] = round(lay / extras["rank0_layer_ms"] - 1, 4)
+        extras["lowrank_overhead_gemm"] = round(k2_ms / extras["rank0_gemm_ms"] - 1, 4)
+        extras["unfused_overhead_layer"] = round(extras["unfused_layer_ms"] / extras["rank0_layer_ms"] - 1, 4)
+
+        # end to end through the public API with host buffers: pinned X in, Y out
+        X_host = X_cpu.pin_memory()
+        Y_host = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step(ev):
+            ev[0].record(stream)
+            X.copy_(X_host, non_blocking=True)
+            S.svdq_quantize_act(X, P.inv_lam, P.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
+            S.svdq_linear(Qx, Sx, T, P, S.SVDQ_FUSED, out=Y)
+            Y_host.copy_(Y, non_blocking=True)
+            ev[1].record(stream)
+            ev[2].record(stream)
+        ke, _ = timed(n_x, e2e_step)
+        e2e_ms = aggregate_max(sum(ke), world) / n_x
+        e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
+               "ms_per_step": round(e2e_ms, 4)}
+        S.svdq_check()
+
+        if rank_id == 0 and world == 1:
+            fn, fl, sample = oracle_sample(w, X_cpu, W_cpu)
+            v, n, el = time_cpu(fn, fl, args.cpu_seconds)
+            cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+                   "sample": sample, "repeats": n, "seconds": round(el, 2)}
+
+    if rank_id == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "M_per_gpu": w.M, "K": w.K, "N": w.N, "rank": w.rank, "alpha": w.alpha,
+                       "global_tokens": w.M * world, "parallelism": f"token-parallel x{world} (weights replicated)",
+                       "l2": "flushed between steps (256 MiB write)"},
+            "roofline": roofline, "roofline_quantize": roofline_q,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
+            "extras": extras, "kernel_src": kernel_source_hash(),
+        }
+        print(json.dumps(line), flush=True)
+        if args.extra_json:
+            with open(args.extra_json, "a") as f:
+                f.write(json.dumps(line) + "\n")
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
