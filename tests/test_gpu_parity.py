@@ -34,11 +34,14 @@ def _inputs(M, K, N, rank, seed, outliers="first4"):
 
 
 CASES = [
-    # M, K, N, rank
+    # M, K, N, rank        N % 256 == 0 runs the CTA-pair GEMM, otherwise the single-CTA one
     (256, 512, 512, 16),      # the tiny layer
     (200, 384, 256, 32),      # ragged M, K % 256 == 128
     (1, 128, 128, 0),         # one row, no branch
+    (1, 256, 256, 16),        # one row on a CTA pair: the second CTA's rows are all past M
     (130, 256, 384, 128),     # maximum rank, ragged M
+    (130, 256, 512, 128),     # maximum rank, ragged M, CTA pair
+    (300, 384, 768, 32),      # ragged M and K on a CTA pair
     (512, 1024, 640, 48),
 ]
 

@@ -12,6 +12,7 @@
 
 #include "svdq.h"
 #include "svdq_gemm.cuh"
+#include "svdq_gemm_pair.cuh"
 #include "svdq_prepare.cuh"
 #include "svdq_quant.cuh"
 #include "svdq_svd.cuh"
@@ -121,6 +122,23 @@ svdq_status make_tmap(CUtensorMap* tm, const void* base, CUtensorMapDataType dt,
   return SVDQ_OK;
 }
 
+// Native scale buffer of `rows` (padded to 128) x K viewed as 4-D uint8
+// [row blocks][K/64 atoms][32 lines][16 bytes]; box of `blocks` row blocks x 4 atoms.
+svdq_status make_scale_tmap(CUtensorMap* tm, const void* base, int64_t rows, int64_t K, uint32_t blocks) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const uint64_t rb = (uint64_t)((rows + 127) / 128), atoms = (uint64_t)(K / 64);
+  const cuuint64_t dims[4] = {16, 32, atoms, rb};
+  const cuuint64_t strides[3] = {16, 512, atoms * 512};
+  const cuuint32_t box[4] = {16, 32, 4, blocks};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);
+  return SVDQ_OK;
+}
+
 size_t scale_bytes(int64_t rows, int64_t K) { return (size_t)((rows + 127) / 128) * (size_t)(K / 64) * 512u; }
 
 // ---------------------------------------------------------------- launchers
@@ -154,53 +172,143 @@ svdq_status launch_quant(const svdq_shape& s, int rank, const void* X, const flo
   }
 }
 
-template <int STAGES, int RANK>
-svdq_status launch_gemm_t(const svdq_shape& s, const CUtensorMap& tqx, const CUtensorMap& tqr, const CUtensorMap& tt,
-                          const CUtensorMap& tl, const void* Sx, const void* Sr, void* Y, cudaStream_t st) {
-  using L = svdq::GemmSmem<STAGES, RANK>;
-  auto kern = svdq::svdq_gemm_kernel<STAGES, RANK>;
-  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
-  dim3 grid((unsigned)(s.N / svdq::kGemmBN), (unsigned)((s.M + svdq::kGemmBM - 1) / svdq::kGemmBM));
-  kern<<<grid, svdq::kGemmThreads, L::kBytes, st>>>(tqx, tqr, tt, tl, static_cast<const uint8_t*>(Sx),
-                                                    static_cast<const uint8_t*>(Sr), static_cast<__nv_bfloat16*>(Y),
-                                                    (int)s.M, (int)s.N, (int)s.K);
-  SVDQ_LAUNCHED("svdq_gemm_kernel");
-  return SVDQ_OK;
+int sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
 }
 
-constexpr int kGemmStages = 4;
+constexpr int kGemmStages = 3;
 
-svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
-                        const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
-  CUtensorMap tqx, tqr, tt, tl;
+svdq_status launch_gemm_single(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T,
+                               const void* Qr, const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+  CUtensorMap tqx, tqr, tt, tl, ty;
   svdq_status r;
-  if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, 128, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+  if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, svdq::kGemmBKBytes,
+                     svdq::kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
     return r;
-  if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.N, 128, 128,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+  if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.N, svdq::kGemmBKBytes,
+                     svdq::kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
     return r;
   if (rank > 0) {
-    if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.M, 16, 128,
-                       CU_TENSOR_MAP_SWIZZLE_32B)) != SVDQ_OK)
+    if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.M, svdq::kGemmLrK,
+                       svdq::kGemmBM, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
       return r;
-    if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.N, 16, 128,
-                       CU_TENSOR_MAP_SWIZZLE_32B)) != SVDQ_OK)
+    if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.N, svdq::kGemmLrK,
+                       svdq::kGemmBN, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
       return r;
   } else {
     memset(&tt, 0, sizeof(tt));
     memset(&tl, 0, sizeof(tl));
   }
-  switch (rank) {
-#define SVDQ_CASE(R) \
-  case R:            \
-    return launch_gemm_t<kGemmStages, R>(s, tqx, tqr, tt, tl, Sx, Sr, Y, st);
-    SVDQ_CASE(0) SVDQ_CASE(16) SVDQ_CASE(32) SVDQ_CASE(48) SVDQ_CASE(64) SVDQ_CASE(80) SVDQ_CASE(96)
-    SVDQ_CASE(112) SVDQ_CASE(128)
-#undef SVDQ_CASE
-    default:
-      return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d", rank);
+  if ((r = make_tmap(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)s.M, svdq::kEpiBoxCols, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  using L = svdq::GemmSmem<kGemmStages>;
+  auto kern = svdq::svdq_gemm_kernel<kGemmStages>;
+  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  const long long tiles = ((s.M + svdq::kGemmBM - 1) / svdq::kGemmBM) * ((s.N + svdq::kGemmBN - 1) / svdq::kGemmBN);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  kern<<<grid, svdq::kGemmThreads, L::kBytes, st>>>(tqx, tqr, tt, tl, ty, static_cast<const uint8_t*>(Sx),
+                                                   static_cast<const uint8_t*>(Sr), (int)s.M, (int)s.N, (int)s.K,
+                                                   rank);
+  SVDQ_LAUNCHED("svdq_gemm_kernel");
+  return SVDQ_OK;
+}
+
+constexpr int kPairStages = 5;
+
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = svdq::PairSmem<kPairStages>::kBytes;
+  cfg.stream = st;
+  attr->id = cudaLaunchAttributeClusterDimension;
+  attr->val.clusterDim.x = 2;
+  attr->val.clusterDim.y = 1;
+  attr->val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+// Clusters of the pair kernel that fit on the device at once (cached per device).
+int pair_clusters() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  auto kern = svdq::svdq_gemm_pair_kernel<kPairStages>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairSmem<kPairStages>::kBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
   }
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t cfg = pair_config(sm_count() / 2, nullptr, &attr);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T,
+                             const void* Qr, const void* Sr, const void* L2t, void* Y, cudaStream_t st,
+                             int clusters) {
+  CUtensorMap tqx, tqr, tsa, tsb, tt, tl, ty;
+  svdq_status r;
+  if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, svdq::kGemmBKBytes,
+                     128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.N, svdq::kGemmBKBytes,
+                     128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if ((r = make_scale_tmap(&tsa, Sx, s.M, s.K, 1)) != SVDQ_OK) return r;
+  if ((r = make_scale_tmap(&tsb, Sr, s.N, s.K, 2)) != SVDQ_OK) return r;
+  if (rank > 0) {
+    if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.M, svdq::kGemmLrK, 128,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+    if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.N, svdq::kGemmLrK,
+                       128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+  } else {
+    memset(&tt, 0, sizeof(tt));
+    memset(&tl, 0, sizeof(tl));
+  }
+  if ((r = make_tmap(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)s.M, svdq::kEpiBoxCols, 32,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  using L = svdq::PairSmem<kPairStages>;
+  auto kern = svdq::svdq_gemm_pair_kernel<kPairStages>;
+  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+  const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / svdq::kPairBN);
+  const int ncl = (int)(tiles < clusters ? tiles : clusters);
+  cudaLaunchAttribute attr;
+  cudaLaunchConfig_t cfg = pair_config(ncl, st, &attr);
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank));
+  SVDQ_LAUNCHED("svdq_gemm_pair_kernel");
+  return SVDQ_OK;
+}
+
+// CTA-pair kernel when N is a multiple of 256 and pairs fit on the device,
+// otherwise the single-CTA kernel.
+svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                        const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+  if (s.N % svdq::kPairBN == 0) {
+    const int clusters = pair_clusters();
+    if (clusters > 0) return launch_gemm_pair(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
+  }
+  return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
 }
 
 template <int RANK>

@@ -7,15 +7,23 @@
 // MMAs (kind::f16) into the same accumulator, so the 16-bit branch adds no pass
 // over Y.
 //
-// One CTA computes one BM x BN = 128 x 128 tile of Y with warp-specialized
-// roles (192 threads):
-//   warps 0-3  epilogue: TMEM -> registers -> bf16 -> global (warp w owns
-//              accumulator lanes 32w..32w+31, i.e. rows m0+32w..)
-//   warp 4     producer: TMA loads of the Qx/Qr tiles (128 B K-rows, 128B
-//              swizzle) and bulk copies of the Sx/Sr scale atoms into a ring
-//              of STAGES shared-memory stages; TMA loads of the T / L2t tiles
-//   warp 5     TMEM allocation; one lane issues tcgen05.cp (scales -> TMEM)
-//              and the MMAs, and commits stage releases / accumulator-ready.
+// This single-CTA kernel serves every N that is a multiple of 128; the CTA-pair
+// kernel (svdq_gemm_pair.cuh) takes over when N is a multiple of 256.
+//
+// Persistent kernel: one CTA per SM walks output tiles of BM x BN = 128 x 256
+// (tile = blockIdx.x, blockIdx.x + gridDim.x, ...). Warp roles (320 threads):
+//   warps 0-7  epilogue: warp w drains accumulator lanes 32(w%4).. and columns
+//              128(w/4).. into registers, releases the accumulator, then
+//              converts to bf16 into a 128B-swizzled shared-memory box and
+//              writes Y with TMA stores (clipped at the matrix edge) while the
+//              next tile's MMAs run
+//   warp 8     producer: per tile, K/256 FP4 k-tiles (TMA loads of 128-byte
+//              K-rows of Qx / Qr with 128B swizzle + bulk copies of the
+//              Sx / Sr scale atoms), then ceil(r/64) low-rank k-tiles (TMA
+//              loads of T and L2t), all through one ring of STAGES stages
+//   warp 9     TMEM allocation; one lane copies scale atoms to TMEM
+//              (tcgen05.cp) and issues the MMAs, releasing each stage with
+//              tcgen05.commit and signalling the epilogue per tile.
 // Every wait is bounded (svdq::mbar_wait); on a timeout the kernel records a
 // device error word and every role drains and returns.
 #pragma once
@@ -27,69 +35,120 @@
 namespace svdq {
 
 constexpr int kGemmBM = 128;
-constexpr int kGemmBN = 128;
-constexpr int kGemmBKBytes = 128;                 // 256 FP4 elements per stage row
-constexpr int kGemmKBPerStage = 4;                // 64-element MMA K blocks per stage
-constexpr int kGemmThreads = 192;
+constexpr int kGemmBN = 256;
+constexpr int kGemmBKBytes = 128;                 // 256 FP4 elements per k-tile row
+constexpr int kGemmKBPerStage = 4;                // 64-element MMA K blocks per k-tile
+constexpr int kGemmEpiWarps = 8;
+constexpr int kGemmThreads = 32 * (kGemmEpiWarps + 2);
+constexpr int kGemmLrK = 64;                      // bf16 K elements per low-rank k-tile
 
-constexpr int kTileABytes = kGemmBM * kGemmBKBytes;   // 16 KB
-constexpr int kTileBBytes = kGemmBN * kGemmBKBytes;   // 16 KB
-constexpr int kSfAtomBytes = 512;                     // 128 rows x 4 scales
+constexpr int kSfAtomBytes = 512;                 // 128 rows x 4 scales
+constexpr int kStageA = kGemmBM * kGemmBKBytes;   // 16 KB (also T: 128 x 64 bf16)
+constexpr int kStageB = kGemmBN * kGemmBKBytes;   // 32 KB (also L2t: 256 x 64 bf16)
+constexpr int kStageSfa = kGemmKBPerStage * kSfAtomBytes;
+constexpr int kStageSfb = 2 * kGemmKBPerStage * kSfAtomBytes;
+constexpr int kStageBytes = kStageA + kStageB + kStageSfa + kStageSfb;   // 54 KB
 
-// TMEM columns: accumulator [0, BN), scale factors of A then B after it.
-constexpr uint32_t kTmemCols = 256;
+// TMEM columns: accumulator [0, 256), then two scale-factor buffers (A scales,
+// then B scales) used by alternate k-tiles.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemSfCols = 4 * kGemmKBPerStage * 3;   // 16 (A) + 32 (B)
 constexpr uint32_t kTmemSfaCol = kGemmBN;
 constexpr uint32_t kTmemSfbCol = kGemmBN + 4 * kGemmKBPerStage;
 
-template <int STAGES, int RANK>
+// Epilogue staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp.
+constexpr int kEpiBoxCols = 64;
+constexpr int kEpiBoxBytes = 32 * kEpiBoxCols * 2;
+
+template <int STAGES>
 struct GemmSmem {
-  static constexpr int kStageBytes = kTileABytes + kTileBBytes + 2 * kGemmKBPerStage * kSfAtomBytes;
-  static constexpr int kLrSlabA = kGemmBM * 32;   // one 16-wide bf16 K slab of T: 128 rows x 32 B
-  static constexpr int kLrSlabB = kGemmBN * 32;
-  static constexpr int kLrBytes = (RANK / 16) * (kLrSlabA + kLrSlabB);
-  static constexpr int kBarOffset = STAGES * kStageBytes + kLrBytes;
+  static constexpr int kEpiOffset = STAGES * kStageBytes;
+  static constexpr int kBarOffset = kEpiOffset + kGemmEpiWarps * kEpiBoxBytes;
   static constexpr int kBytes = kBarOffset + 256 + 1024;   // barriers + alignment slack
 };
 
-template <int STAGES, int RANK>
+// Epilogue of one tile for one warp: `v` holds 128 fp32 accumulator columns of
+// row `lane` of the warp's 32-row band; written as two 32 x 64 bf16 boxes.
+__device__ __forceinline__ void epilogue_store_band(const uint32_t (&v)[128], unsigned char* box, const void* tm_y,
+                                                    int col0, int row0, int lane, bool store) {
+  const uint32_t box_addr = smem_u32(box);
+#pragma unroll
+  for (int b = 0; b < 2; ++b) {
+    if (lane == 0) bulk_wait_read<0>();   // the previous store from this box has read it
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t p[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 64 * b + 8 * c + 2 * i;
+        const __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+        p[i] = *reinterpret_cast<const uint32_t*>(&bb);
+      }
+      // row `lane`: chunk c of 16 B at (c ^ (lane & 7)) -- the 128B swizzle pattern
+      const uint32_t addr = box_addr + lane * 128 + ((c ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0 && store) {
+      tma_store_2d(tm_y, box, col0 + 64 * b, row0);
+      bulk_commit();
+    }
+  }
+}
+
+// Drain 128 accumulator columns of this warp's lane band into registers.
+__device__ __forceinline__ void epilogue_drain(uint32_t taddr, uint32_t (&v)[128]) {
+  tmem_ld_32x32b_x32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
+  tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+  tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
+  tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
+  tmem_ld_wait();
+}
+
+template <int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_qx, const __grid_constant__ CUtensorMap tm_qr,
     const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
-    const uint8_t* __restrict__ Sx, const uint8_t* __restrict__ Sr, __nv_bfloat16* __restrict__ Y, int M, int N,
-    int K) {
-  using L = GemmSmem<STAGES, RANK>;
+    const __grid_constant__ CUtensorMap tm_y, const uint8_t* __restrict__ Sx, const uint8_t* __restrict__ Sr,
+    int M, int N, int K, int rank) {
+  using L = GemmSmem<STAGES>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
-  uint64_t* lr_full = empty + STAGES;
-  uint64_t* acc_full = lr_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_full + 1);
-  unsigned char* lr_a = smem + STAGES * L::kStageBytes;
-  unsigned char* lr_b = lr_a + (RANK / 16) * L::kLrSlabA;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* mma_drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * kGemmBN, m0 = blockIdx.y * kGemmBM;
+  const int tiles_n = (N + kGemmBN - 1) / kGemmBN;
+  const int ntiles = ((M + kGemmBM - 1) / kGemmBM) * tiles_n;
   const int kb_total = K >> 6;
-  const int num_kt = (kb_total + kGemmKBPerStage - 1) / kGemmKBPerStage;
+  const int n_fp4_kt = (kb_total + kGemmKBPerStage - 1) / kGemmKBPerStage;
+  const int n_lr_kt = (rank + kGemmLrK - 1) / kGemmLrK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    mbar_init(lr_full, 1);
     mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kGemmEpiWarps);
+    mbar_init(mma_drain, 1);
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == kGemmEpiWarps + 1) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kGemmEpiWarps && lane == 0) {
     prefetch_tmap(&tm_qx);
     prefetch_tmap(&tm_qr);
-    if (RANK > 0) {
+    if (rank > 0) {
       prefetch_tmap(&tm_t);
       prefetch_tmap(&tm_l2);
     }
@@ -99,120 +158,141 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == kGemmEpiWarps) {
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      if (RANK > 0) {
-        mbar_arrive_expect_tx(lr_full, (uint32_t)L::kLrBytes);
-        for (int j = 0; j < RANK / 16; ++j) {
-          tma_load_2d(lr_a + j * L::kLrSlabA, &tm_t, lr_full, j * 16, m0);
-          tma_load_2d(lr_b + j * L::kLrSlabB, &tm_l2, lr_full, j * 16, n0);
+      // ---------------------------------------------------------------- producer
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+        const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+        const bool half = n0 + kGemmBN > N;    // only the first 128 B rows exist
+        const uint8_t* sfa_src = Sx + (size_t)(m0 >> 7) * kb_total * kSfAtomBytes;
+        const uint8_t* sfb_src = Sr + (size_t)(n0 >> 7) * kb_total * kSfAtomBytes;
+        for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(empty + s, ((it / STAGES) & 1u) ^ 1u, kDevErrTimeoutEmpty)) {
+            ok = false;
+            break;
+          }
+          unsigned char* sa = smem + s * kStageBytes;
+          unsigned char* sb = sa + kStageA;
+          if (kt < n_fp4_kt) {
+            unsigned char* sfa = sb + kStageB;
+            unsigned char* sfb = sfa + kStageSfa;
+            const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
+            const uint32_t sf_bytes = (uint32_t)kbs * kSfAtomBytes;
+            mbar_arrive_expect_tx(full + s, (uint32_t)(kStageA + kStageB) + sf_bytes * (half ? 2u : 3u));
+            tma_load_2d(sa, &tm_qx, full + s, kt * kGemmBKBytes, m0);
+            tma_load_2d(sb, &tm_qr, full + s, kt * kGemmBKBytes, n0);
+            const size_t off = (size_t)kt * kGemmKBPerStage * kSfAtomBytes;
+            bulk_load(sfa, sfa_src + off, sf_bytes, full + s);
+            bulk_load(sfb, sfb_src + off, sf_bytes, full + s);
+            if (!half)
+              bulk_load(sfb + kStageSfb / 2, sfb_src + (size_t)kb_total * kSfAtomBytes + off, sf_bytes, full + s);
+          } else {
+            const int c = kt - n_fp4_kt;
+            mbar_arrive_expect_tx(full + s, (uint32_t)(kStageA + kStageB));
+            tma_load_2d(sa, &tm_t, full + s, c * kGemmLrK, m0);
+            tma_load_2d(sb, &tm_l2, full + s, c * kGemmLrK, n0);
+          }
         }
-      }
-      const uint8_t* sfa_src = Sx + (size_t)(m0 >> 7) * kb_total * kSfAtomBytes;
-      const uint8_t* sfb_src = Sr + (size_t)(n0 >> 7) * kb_total * kSfAtomBytes;
-      for (int kt = 0; kt < num_kt; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-        if (!mbar_wait(empty + s, ph ^ 1u, kDevErrTimeoutEmpty)) break;
-        const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
-        unsigned char* st = smem + s * L::kStageBytes;
-        unsigned char* sa = st;
-        unsigned char* sb = st + kTileABytes;
-        unsigned char* sfa = sb + kTileBBytes;
-        unsigned char* sfb = sfa + kGemmKBPerStage * kSfAtomBytes;
-        mbar_arrive_expect_tx(full + s, (uint32_t)(kTileABytes + kTileBBytes + 2 * kbs * kSfAtomBytes));
-        tma_load_2d(sa, &tm_qx, full + s, kt * kGemmBKBytes, m0);
-        tma_load_2d(sb, &tm_qr, full + s, kt * kGemmBKBytes, n0);
-        bulk_load(sfa, sfa_src + (size_t)kt * kGemmKBPerStage * kSfAtomBytes, kbs * kSfAtomBytes, full + s);
-        bulk_load(sfb, sfb_src + (size_t)kt * kGemmKBPerStage * kSfAtomBytes, kbs * kSfAtomBytes, full + s);
       }
       if (device_error_set()) {
         // Another role gave up: let the copies this thread issued land before
-        // the CTA exits (bounded; the stages of the last STAGES k-tiles and
-        // the low-rank tiles are the only ones that can still be in flight).
-        for (int kt = max(0, num_kt - STAGES); kt < num_kt; ++kt)
-          mbar_wait(full + kt % STAGES, (uint32_t)(kt / STAGES) & 1u, kDevErrTimeoutFull);
-        if (RANK > 0) mbar_wait(lr_full, 0, kDevErrTimeoutFull);
+        // the CTA exits (bounded; only the last STAGES stages can be in flight).
+        for (uint32_t j = it > (uint32_t)STAGES ? it - STAGES : 0u; j < it; ++j)
+          mbar_wait(full + j % STAGES, (j / STAGES) & 1u, kDevErrTimeoutFull);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == kGemmEpiWarps + 1) {
     if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      const uint32_t idesc = idesc_nvfp4(kGemmBM, kGemmBN);
+      // ---------------------------------------------------------------- MMA issuer
+      uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int kt = 0; kt < num_kt && ok; ++kt) {
-        const int s = kt % STAGES;
-        const uint32_t ph = (uint32_t)(kt / STAGES) & 1u;
-        if (!mbar_wait(full + s, ph, kDevErrTimeoutFull)) {
+      for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++tcount) {
+        const int n0 = (tile % tiles_n) * kGemmBN;
+        const bool half = n0 + kGemmBN > N;
+        const uint32_t idesc = idesc_nvfp4(kGemmBM, half ? kGemmBN / 2 : kGemmBN);
+        const uint32_t idesc_lr = idesc_bf16(kGemmBM, half ? kGemmBN / 2 : kGemmBN);
+        if (!mbar_wait(acc_empty, (tcount & 1u) ^ 1u, kDevErrTimeoutAccum)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
-        unsigned char* st = smem + s * L::kStageBytes;
-        const uint32_t sa = smem_u32(st);
-        const uint32_t sb = sa + kTileABytes;
-        const uint32_t sfa = sb + kTileBBytes;
-        const uint32_t sfb = sfa + kGemmKBPerStage * kSfAtomBytes;
-        for (int kb = 0; kb < kbs; ++kb) {
-          tmem_cp_32x128b_x4(tmem + kTmemSfaCol + 4 * kb, smem_desc(sfa + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
-          tmem_cp_32x128b_x4(tmem + kTmemSfbCol + 4 * kb, smem_desc(sfb + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
-        }
-        for (int kb = 0; kb < kbs; ++kb) {
-          const uint64_t ad = smem_desc(sa + kb * 32, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(sb + kb * 32, 16, 1024, kSwizzle128B);
-          mma_nvfp4(tmem, ad, bd, idesc, tmem + kTmemSfaCol + 4 * kb, tmem + kTmemSfbCol + 4 * kb,
-                    (kt | kb) != 0 ? 1u : 0u);
-        }
-        tc_commit(empty + s);   // stage s is free once these MMAs have read it
-      }
-      if (ok && RANK > 0) {
-        if (mbar_wait(lr_full, 0, kDevErrTimeoutFull)) {
-          tc_fence_after();
-          const uint32_t idl = idesc_bf16(kGemmBM, kGemmBN);
-          const uint32_t la = smem_u32(lr_a), lb = smem_u32(lr_b);
-          for (int j = 0; j < RANK / 16; ++j) {
-            const uint64_t ad = smem_desc(la + j * L::kLrSlabA, 16, 256, kSwizzle32B);
-            const uint64_t bd = smem_desc(lb + j * L::kLrSlabB, 16, 256, kSwizzle32B);
-            mma_bf16(tmem, ad, bd, idl, (num_kt > 0 || j > 0) ? 1u : 0u);
+        for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull)) {
+            ok = false;
+            break;
           }
-        } else {
-          ok = false;
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + s * kStageBytes);
+          const uint32_t sb = sa + kStageA;
+          if (kt < n_fp4_kt) {
+            const uint32_t sfa = sb + kStageB;
+            const uint32_t sfb = sfa + kStageSfa;
+            const uint32_t col = (it & 1u) * kTmemSfCols;   // alternate scale buffers
+            const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
+            for (int kb = 0; kb < kbs; ++kb) {
+              tmem_cp_32x128b_x4(tmem + kTmemSfaCol + col + 4 * kb,
+                                 smem_desc(sfa + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
+              tmem_cp_32x128b_x4(tmem + kTmemSfbCol + col + 8 * kb,
+                                 smem_desc(sfb + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
+              if (!half)
+                tmem_cp_32x128b_x4(tmem + kTmemSfbCol + col + 8 * kb + 4,
+                                   smem_desc(sfb + kStageSfb / 2 + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
+            }
+            for (int kb = 0; kb < kbs; ++kb) {
+              const uint64_t ad = smem_desc(sa + kb * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(sb + kb * 32, 16, 1024, kSwizzle128B);
+              mma_nvfp4(tmem, ad, bd, idesc, tmem + kTmemSfaCol + col + 4 * kb, tmem + kTmemSfbCol + col + 8 * kb,
+                        (kt | kb) != 0 ? 1u : 0u);
+            }
+          } else {
+            const int c = kt - n_fp4_kt;
+            const int k16 = min(kGemmLrK, rank - c * kGemmLrK) / 16;
+            for (int j = 0; j < k16; ++j) {
+              const uint64_t ad = smem_desc(sa + j * 32, 16, 1024, kSwizzle128B);
+              const uint64_t bd = smem_desc(sb + j * 32, 16, 1024, kSwizzle128B);
+              mma_bf16(tmem, ad, bd, idesc_lr, 1u);
+            }
+          }
+          tc_commit(empty + s);   // stage s is free once these MMAs have read it
         }
+        tc_commit(acc_full);      // the tile's accumulator is complete
       }
-      tc_commit(acc_full);   // arrives when every MMA above has completed
+      if (!ok) {
+        // Gave up: wait (bounded) for the MMAs already issued before TMEM is freed.
+        tc_commit(mma_drain);
+        mbar_wait(mma_drain, 0, kDevErrTimeoutAccum);
+      }
     }
   } else {
-    // -------------------------------------------------------------- epilogue
-    const bool ok = mbar_wait(acc_full, 0, kDevErrTimeoutAccum);
-    tc_fence_after();
-    if (ok && !device_error_set()) {
-      const int row = m0 + warp * 32 + lane;
-      const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-#pragma unroll 1
-      for (int c = 0; c < kGemmBN; c += 32) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(lane_addr + c, v);
-        tmem_ld_wait();
-        if (row < M) {
-          uint32_t p[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 b = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            p[i] = *reinterpret_cast<const uint32_t*>(&b);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * N + n0 + c);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
-        }
-      }
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3, h = warp >> 2;
+    unsigned char* box = smem + L::kEpiOffset + warp * kEpiBoxBytes;
+    if (lane == 0) prefetch_tmap(&tm_y);
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++tcount) {
+      const int m0 = (tile / tiles_n) * kGemmBM, n0 = (tile % tiles_n) * kGemmBN;
+      const bool ok = mbar_wait(acc_full, tcount & 1u, kDevErrTimeoutAccum);
+      tc_fence_after();
+      if (!ok || device_error_set()) break;
+      uint32_t v[128];
+      epilogue_drain(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);   // accumulator drained: the next tile may start
+      const int col0 = n0 + h * 128;
+      if (col0 >= N) continue;                 // second half of a 128-wide last column tile
+      epilogue_store_band(v, box, &tm_y, col0, m0 + 32 * q, lane, true);
     }
+    if (lane == 0) bulk_wait<0>();   // every store of this warp has completed
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kGemmEpiWarps + 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
