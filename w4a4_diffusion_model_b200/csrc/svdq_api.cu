@@ -122,17 +122,18 @@ svdq_status make_tmap(CUtensorMap* tm, const void* base, CUtensorMapDataType dt,
   return SVDQ_OK;
 }
 
-// Native scale buffer of `rows` (padded to 128) x K viewed as 4-D uint8
-// [row blocks][K/64 atoms][32 lines][16 bytes]; box of `blocks` row blocks x 4 atoms.
+// Native scale buffer of `rows` (padded to 128) x K viewed as 3-D uint8
+// [row blocks][K/64 * 2 chunks][256 bytes] (the atoms of one row block are
+// contiguous, 512 bytes each); box of `blocks` row blocks x 8 chunks = 4 atoms.
 svdq_status make_scale_tmap(CUtensorMap* tm, const void* base, int64_t rows, int64_t K, uint32_t blocks) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const uint64_t rb = (uint64_t)((rows + 127) / 128), atoms = (uint64_t)(K / 64);
-  const cuuint64_t dims[4] = {16, 32, atoms, rb};
-  const cuuint64_t strides[3] = {16, 512, atoms * 512};
-  const cuuint32_t box[4] = {16, 32, 4, blocks};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides, box, estr,
+  const uint64_t rb = (uint64_t)((rows + 127) / 128), chunks = (uint64_t)(K / 64) * 2;
+  const cuuint64_t dims[3] = {256, chunks, rb};
+  const cuuint64_t strides[2] = {256, chunks * 256};
+  const cuuint32_t box[3] = {256, 8, blocks};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(SVDQ_ERR_CUDA, "cuTensorMapEncodeTiled (scales) failed (%d)", (int)r);

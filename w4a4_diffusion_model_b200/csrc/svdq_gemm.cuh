@@ -11,102 +11,44 @@
 // kernel (svdq_gemm_pair.cuh) takes over when N is a multiple of 256.
 //
 // Persistent kernel: one CTA per SM walks output tiles of BM x BN = 128 x 256
-// (tile = blockIdx.x, blockIdx.x + gridDim.x, ...). Warp roles (320 threads):
-//   warps 0-7  epilogue: warp w drains accumulator lanes 32(w%4).. and columns
-//              128(w/4).. into registers, releases the accumulator, then
-//              converts to bf16 into a 128B-swizzled shared-memory box and
-//              writes Y with TMA stores (clipped at the matrix edge) while the
-//              next tile's MMAs run
-//   warp 8     producer: per tile, K/256 FP4 k-tiles (TMA loads of 128-byte
-//              K-rows of Qx / Qr with 128B swizzle + bulk copies of the
-//              Sx / Sr scale atoms), then ceil(r/64) low-rank k-tiles (TMA
-//              loads of T and L2t), all through one ring of STAGES stages
-//   warp 9     TMEM allocation; one lane copies scale atoms to TMEM
-//              (tcgen05.cp) and issues the MMAs, releasing each stage with
-//              tcgen05.commit and signalling the epilogue per tile.
+// (tile = blockIdx.x, blockIdx.x + gridDim.x, ...). Every tile is a sequence
+// of k-tiles ("items"): K/256 FP4 items, then ceil(r/64) low-rank items, all
+// through one ring of STAGES shared-memory stages. Warp roles (448 threads):
+//   warps 0-7   epilogue: warp w drains accumulator lanes 32(w%4).. and columns
+//               128(w/4).., releases the accumulator, then writes Y through
+//               128B-swizzled boxes and TMA stores while the next tile runs
+//   warp 8      producer: TMA loads of the Qx / Qr (then T / L2t) k-tile rows
+//               and bulk copies of the Sx / Sr scale atoms into the ring
+//   warp 9      TMEM allocation; one lane issues the MMAs of each item once its
+//               scales are in TMEM, and releases ring stages, scale buffers
+//               and the accumulator with tcgen05.commit
+//   warps 10-13 scale warps: copy each item's scale atoms into a TMEM scale
+//               buffer with tcgen05.st (svdq_gemm_common.cuh)
 // Every wait is bounded (svdq::mbar_wait); on a timeout the kernel records a
 // device error word and every role drains and returns.
 #pragma once
 
 #include <cuda_bf16.h>
 
+#include "svdq_gemm_common.cuh"
 #include "svdq_ptx.cuh"
 
 namespace svdq {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBN = 256;
-constexpr int kGemmBKBytes = 128;                 // 256 FP4 elements per k-tile row
-constexpr int kGemmKBPerStage = 4;                // 64-element MMA K blocks per k-tile
-constexpr int kGemmEpiWarps = 8;
-constexpr int kGemmThreads = 32 * (kGemmEpiWarps + 2);
-constexpr int kGemmLrK = 64;                      // bf16 K elements per low-rank k-tile
-
-constexpr int kSfAtomBytes = 512;                 // 128 rows x 4 scales
 constexpr int kStageA = kGemmBM * kGemmBKBytes;   // 16 KB (also T: 128 x 64 bf16)
 constexpr int kStageB = kGemmBN * kGemmBKBytes;   // 32 KB (also L2t: 256 x 64 bf16)
 constexpr int kStageSfa = kGemmKBPerStage * kSfAtomBytes;
 constexpr int kStageSfb = 2 * kGemmKBPerStage * kSfAtomBytes;
 constexpr int kStageBytes = kStageA + kStageB + kStageSfa + kStageSfb;   // 54 KB
 
-// TMEM columns: accumulator [0, 256), then two scale-factor buffers (A scales,
-// then B scales) used by alternate k-tiles.
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfCols = 4 * kGemmKBPerStage * 3;   // 16 (A) + 32 (B)
-constexpr uint32_t kTmemSfaCol = kGemmBN;
-constexpr uint32_t kTmemSfbCol = kGemmBN + 4 * kGemmKBPerStage;
-
-// Epilogue staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp.
-constexpr int kEpiBoxCols = 64;
-constexpr int kEpiBoxBytes = 32 * kEpiBoxCols * 2;
-
 template <int STAGES>
 struct GemmSmem {
   static constexpr int kEpiOffset = STAGES * kStageBytes;
   static constexpr int kBarOffset = kEpiOffset + kGemmEpiWarps * kEpiBoxBytes;
-  static constexpr int kBytes = kBarOffset + 256 + 1024;   // barriers + alignment slack
+  static constexpr int kBytes = kBarOffset + 512 + 1024;   // barriers + alignment slack
 };
-
-// Epilogue of one tile for one warp: `v` holds 128 fp32 accumulator columns of
-// row `lane` of the warp's 32-row band; written as two 32 x 64 bf16 boxes.
-__device__ __forceinline__ void epilogue_store_band(const uint32_t (&v)[128], unsigned char* box, const void* tm_y,
-                                                    int col0, int row0, int lane, bool store) {
-  const uint32_t box_addr = smem_u32(box);
-#pragma unroll
-  for (int b = 0; b < 2; ++b) {
-    if (lane == 0) bulk_wait_read<0>();   // the previous store from this box has read it
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t p[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int e = 64 * b + 8 * c + 2 * i;
-        const __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
-        p[i] = *reinterpret_cast<const uint32_t*>(&bb);
-      }
-      // row `lane`: chunk c of 16 B at (c ^ (lane & 7)) -- the 128B swizzle pattern
-      const uint32_t addr = box_addr + lane * 128 + ((c ^ (lane & 7)) << 4);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[0]), "r"(p[1]), "r"(p[2]), "r"(p[3])
-                   : "memory");
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0 && store) {
-      tma_store_2d(tm_y, box, col0 + 64 * b, row0);
-      bulk_commit();
-    }
-  }
-}
-
-// Drain 128 accumulator columns of this warp's lane band into registers.
-__device__ __forceinline__ void epilogue_drain(uint32_t taddr, uint32_t (&v)[128]) {
-  tmem_ld_32x32b_x32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(v + 0));
-  tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
-  tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(v + 64));
-  tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(v + 96));
-  tmem_ld_wait();
-}
 
 template <int STAGES>
 __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
@@ -119,7 +61,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
-  uint64_t* acc_full = empty + STAGES;
+  uint64_t* sf_ready = empty + STAGES;
+  uint64_t* sf_free = sf_ready + kSfBufs;
+  uint64_t* acc_full = sf_free + kSfBufs;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
@@ -136,16 +80,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
+    for (int b = 0; b < kSfBufs; ++b) {
+      mbar_init(sf_ready + b, kSfWarps);
+      mbar_init(sf_free + b, 1);
+    }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kGemmEpiWarps);
     mbar_init(mma_drain, 1);
     fence_mbar_init();
   }
-  if (warp == kGemmEpiWarps + 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == kGemmEpiWarps && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tm_qx);
     prefetch_tmap(&tm_qr);
     if (rank > 0) {
@@ -158,7 +106,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kGemmEpiWarps) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       uint32_t it = 0;
@@ -204,7 +152,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
           mbar_wait(full + j % STAGES, (j / STAGES) & 1u, kDevErrTimeoutFull);
       }
     }
-  } else if (warp == kGemmEpiWarps + 1) {
+  } else if (warp >= kSfWarp0) {
+    // ------------------------------------------------------------------ scale warps
+    const int q = warp & 3;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+      for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
+        const int s = it % STAGES, b = it % kSfBufs;
+        if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull) ||
+            (it >= (uint32_t)kSfBufs && !mbar_wait(sf_free + b, ((it / kSfBufs) - 1u) & 1u, kDevErrTimeoutScales))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (kt < n_fp4_kt) {
+          const unsigned char* sfa = smem + s * kStageBytes + kStageA + kStageB;
+          const unsigned char* sfb = sfa + kStageSfa;
+          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kStageSfb / 2, sf_buf_col(b));
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sf_ready + b);
+      }
+    }
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       // ---------------------------------------------------------------- MMA issuer
       uint32_t it = 0, tcount = 0;
@@ -220,8 +193,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
         }
         tc_fence_after();
         for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-          const int s = it % STAGES;
-          if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull)) {
+          const int s = it % STAGES, b = it % kSfBufs;
+          // the scale warps saw stage s full and put its scales in buffer b
+          if (!mbar_wait(sf_ready + b, (it / kSfBufs) & 1u, kDevErrTimeoutScales)) {
             ok = false;
             break;
           }
@@ -229,24 +203,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
           const uint32_t sa = smem_u32(smem + s * kStageBytes);
           const uint32_t sb = sa + kStageA;
           if (kt < n_fp4_kt) {
-            const uint32_t sfa = sb + kStageB;
-            const uint32_t sfb = sfa + kStageSfa;
-            const uint32_t col = (it & 1u) * kTmemSfCols;   // alternate scale buffers
+            const uint32_t sfa = tmem + sf_buf_col(b);
+            const uint32_t sfb = sfa + 4 * kGemmKBPerStage;
             const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
-            for (int kb = 0; kb < kbs; ++kb) {
-              tmem_cp_32x128b_x4(tmem + kTmemSfaCol + col + 4 * kb,
-                                 smem_desc(sfa + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
-              tmem_cp_32x128b_x4(tmem + kTmemSfbCol + col + 8 * kb,
-                                 smem_desc(sfb + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
-              if (!half)
-                tmem_cp_32x128b_x4(tmem + kTmemSfbCol + col + 8 * kb + 4,
-                                   smem_desc(sfb + kStageSfb / 2 + kb * kSfAtomBytes, 16, 128, kSwizzleNone));
-            }
             for (int kb = 0; kb < kbs; ++kb) {
               const uint64_t ad = smem_desc(sa + kb * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(sb + kb * 32, 16, 1024, kSwizzle128B);
-              mma_nvfp4(tmem, ad, bd, idesc, tmem + kTmemSfaCol + col + 4 * kb, tmem + kTmemSfbCol + col + 8 * kb,
-                        (kt | kb) != 0 ? 1u : 0u);
+              mma_nvfp4(tmem, ad, bd, idesc, sfa + 4 * kb, sfb + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
             }
           } else {
             const int c = kt - n_fp4_kt;
@@ -257,9 +220,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
               mma_bf16(tmem, ad, bd, idesc_lr, 1u);
             }
           }
-          tc_commit(empty + s);   // stage s is free once these MMAs have read it
+          tc_commit(empty + s);     // ring stage s is free once these MMAs have read it
+          tc_commit(sf_free + b);   // and so is scale buffer b
         }
-        tc_commit(acc_full);      // the tile's accumulator is complete
+        tc_commit(acc_full);        // the tile's accumulator is complete
       }
       if (!ok) {
         // Gave up: wait (bounded) for the MMAs already issued before TMEM is freed.
@@ -278,21 +242,21 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
       const bool ok = mbar_wait(acc_full, tcount & 1u, kDevErrTimeoutAccum);
       tc_fence_after();
       if (!ok || device_error_set()) break;
-      uint32_t v[128];
-      epilogue_drain(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), v);
+      uint32_t p[64];
+      epilogue_drain_pack(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), p);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);   // accumulator drained: the next tile may start
       const int col0 = n0 + h * 128;
       if (col0 >= N) continue;                 // second half of a 128-wide last column tile
-      epilogue_store_band(v, box, &tm_y, col0, m0 + 32 * q, lane, true);
+      epilogue_store_band(p, box, &tm_y, col0, m0 + 32 * q, lane, true);
     }
     if (lane == 0) bulk_wait<0>();   // every store of this warp has completed
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kGemmEpiWarps + 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
