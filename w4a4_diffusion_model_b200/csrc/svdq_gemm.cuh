@@ -20,10 +20,10 @@
 //   warp 8      producer: TMA loads of the Qx / Qr (then T / L2t) k-tile rows
 //               and bulk copies of the Sx / Sr scale atoms into the ring
 //   warp 9      TMEM allocation; one lane issues the MMAs of each item once its
-//               scales are in TMEM, and releases ring stages, scale buffers
-//               and the accumulator with tcgen05.commit
-//   warps 10-13 scale warps: copy each item's scale atoms into a TMEM scale
-//               buffer with tcgen05.st (svdq_gemm_common.cuh)
+//               scales are in TMEM, and releases each ring stage (with its
+//               TMEM scale buffer) and the accumulator with tcgen05.commit
+//   warps 10-13 scale warps: copy each item's scale atoms into the TMEM scale
+//               buffer of its ring stage with tcgen05.st (svdq_gemm_common.cuh)
 // Every wait is bounded (svdq::mbar_wait); on a timeout the kernel records a
 // device error word and every role drains and returns.
 #pragma once
@@ -57,13 +57,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
     const __grid_constant__ CUtensorMap tm_y, const uint8_t* __restrict__ Sx, const uint8_t* __restrict__ Sr,
     int M, int N, int K, int rank) {
   using L = GemmSmem<STAGES>;
+  static_assert(STAGES <= kMaxSfBufs, "one TMEM scale buffer per ring stage");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_ready = empty + STAGES;
-  uint64_t* sf_free = sf_ready + kSfBufs;
-  uint64_t* acc_full = sf_free + kSfBufs;
+  uint64_t* acc_full = sf_ready + STAGES;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* mma_drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
@@ -80,10 +80,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < kSfBufs; ++b) {
-      mbar_init(sf_ready + b, kSfWarps);
-      mbar_init(sf_free + b, 1);
-    }
+    for (int b = 0; b < STAGES; ++b) mbar_init(sf_ready + b, kSfWarps);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kGemmEpiWarps);
     mbar_init(mma_drain, 1);
@@ -159,9 +156,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
       for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-        const int s = it % STAGES, b = it % kSfBufs;
-        if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull) ||
-            (it >= (uint32_t)kSfBufs && !mbar_wait(sf_free + b, ((it / kSfBufs) - 1u) & 1u, kDevErrTimeoutScales))) {
+        const int s = it % STAGES;
+        // stage s has landed; its scale buffer was freed by the commit that
+        // released the stage's previous use (which preceded this refill)
+        if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull)) {
           ok = false;
           break;
         }
@@ -169,12 +167,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
         if (kt < n_fp4_kt) {
           const unsigned char* sfa = smem + s * kStageBytes + kStageA + kStageB;
           const unsigned char* sfb = sfa + kStageSfa;
-          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kStageSfb / 2, sf_buf_col(b));
+          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kStageSfb / 2, sf_buf_col(s));
           tmem_st_wait();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(sf_ready + b);
+        if (lane == 0) mbar_arrive(sf_ready + s);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -193,9 +191,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
         }
         tc_fence_after();
         for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-          const int s = it % STAGES, b = it % kSfBufs;
-          // the scale warps saw stage s full and put its scales in buffer b
-          if (!mbar_wait(sf_ready + b, (it / kSfBufs) & 1u, kDevErrTimeoutScales)) {
+          const int s = it % STAGES;
+          // the scale warps saw stage s full and put its scales in TMEM
+          if (!mbar_wait(sf_ready + s, (it / STAGES) & 1u, kDevErrTimeoutScales)) {
             ok = false;
             break;
           }
@@ -203,7 +201,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
           const uint32_t sa = smem_u32(smem + s * kStageBytes);
           const uint32_t sb = sa + kStageA;
           if (kt < n_fp4_kt) {
-            const uint32_t sfa = tmem + sf_buf_col(b);
+            const uint32_t sfa = tmem + sf_buf_col(s);
             const uint32_t sfb = sfa + 4 * kGemmKBPerStage;
             const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
             for (int kb = 0; kb < kbs; ++kb) {
@@ -220,8 +218,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
               mma_bf16(tmem, ad, bd, idesc_lr, 1u);
             }
           }
-          tc_commit(empty + s);     // ring stage s is free once these MMAs have read it
-          tc_commit(sf_free + b);   // and so is scale buffer b
+          tc_commit(empty + s);     // ring stage s and its scale buffer are free once these MMAs ran
         }
         tc_commit(acc_full);        // the tile's accumulator is complete
       }

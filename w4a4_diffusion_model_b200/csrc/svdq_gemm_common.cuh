@@ -7,8 +7,8 @@
 // issuing thread waits for those copies; the MMA issuer would then idle for a
 // large part of every k-tile. Instead four warps (one per TMEM lane quadrant)
 // load each k-tile's scale atoms from shared memory and write them with
-// tcgen05.st into one of kSfBufs rotating TMEM buffers, and the MMA issuer
-// only ever waits for "scales ready" and "accumulator free".
+// tcgen05.st into the TMEM scale buffer of the item's ring stage, and the MMA
+// issuer only ever waits for "scales ready" and "accumulator free".
 #pragma once
 
 #include <cuda_bf16.h>
@@ -30,12 +30,14 @@ constexpr int kSfWarp0 = 10;
 constexpr int kSfWarps = 4;
 constexpr int kGemmThreads = 32 * (kGemmEpiWarps + 2 + kSfWarps);
 
-// TMEM: accumulator columns [0, 256); then kSfBufs scale buffers of 48 columns:
-// A scales (4 columns per K block) then B scales (8 columns per K block).
+// TMEM: accumulator columns [0, 256); then one scale buffer of 48 columns per
+// ring stage (A scales: 4 columns per K block, then B scales: 8 per K block),
+// so that the one tcgen05.commit that frees a ring stage also frees its scale
+// buffer. At most 5 stages fit: 256 + 5 * 48 = 496 <= 512 columns.
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = 256;
-constexpr int kSfBufs = 4;
 constexpr uint32_t kSfBufCols = 4 * kGemmKBPerStage + 8 * kGemmKBPerStage;
+constexpr int kMaxSfBufs = (int)((kTmemCols - kAccCols) / kSfBufCols);
 __host__ __device__ constexpr uint32_t sf_buf_col(int b) { return kAccCols + (uint32_t)b * kSfBufCols; }
 
 // Epilogue staging: one 32-row x 64-column bf16 box (4 KB) per epilogue warp.

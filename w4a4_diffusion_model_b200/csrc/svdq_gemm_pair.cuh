@@ -18,10 +18,11 @@
 //               counted on this CTA's own stage barrier
 //   warp 9      TMEM allocation (both CTAs); in the even CTA one lane issues
 //               the pair MMAs of each item once both CTAs' scale warps have
-//               reported it, and releases stages, scale buffers and the
-//               accumulator of both CTAs with multicast tcgen05.commit
-//   warps 10-13 scale warps: wait for this CTA's stage, put its scales in a
-//               TMEM scale buffer (tcgen05.st), report to the even CTA
+//               reported it, and releases each ring stage (with its TMEM
+//               scale buffer) and the accumulator of both CTAs with
+//               multicast tcgen05.commit
+//   warps 10-13 scale warps: wait for this CTA's stage, put its scales in the
+//               stage's TMEM scale buffer (tcgen05.st), report to the even CTA
 // Every wait is bounded; on a timeout the kernel records a device error word,
 // every role stops, and both CTAs still meet at the final cluster barrier.
 #pragma once
@@ -58,13 +59,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
     const __grid_constant__ CUtensorMap tm_y, int M, int N, int K, int rank) {
   using L = PairSmem<STAGES>;
+  static_assert(STAGES <= kMaxSfBufs, "one TMEM scale buffer per ring stage");
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_ready = empty + STAGES;      // even CTA: both CTAs' scale warps report here
-  uint64_t* sf_free = sf_ready + kSfBufs;
-  uint64_t* acc_full = sf_free + kSfBufs;
+  uint64_t* acc_full = sf_ready + STAGES;
   uint64_t* acc_empty = acc_full + 1;       // even CTA: both CTAs' epilogue warps report here
   uint64_t* mma_drain = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
@@ -84,10 +85,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
     }
-    for (int b = 0; b < kSfBufs; ++b) {
-      mbar_init(sf_ready + b, 2 * kSfWarps);
-      mbar_init(sf_free + b, 1);
-    }
+    for (int b = 0; b < STAGES; ++b) mbar_init(sf_ready + b, 2 * kSfWarps);
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kGemmEpiWarps);
     mbar_init(mma_drain, 1);
@@ -157,9 +155,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     bool ok = true;
     for (int tile = cluster; tile < ntiles && ok; tile += nclusters) {
       for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-        const int s = it % STAGES, b = it % kSfBufs;
-        if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull) ||
-            (it >= (uint32_t)kSfBufs && !mbar_wait(sf_free + b, ((it / kSfBufs) - 1u) & 1u, kDevErrTimeoutScales))) {
+        const int s = it % STAGES;
+        // stage s has landed; its scale buffer was freed by the commit that
+        // released the stage's previous use (which preceded this refill)
+        if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull)) {
           ok = false;
           break;
         }
@@ -167,12 +166,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         if (kt < n_fp4_kt) {
           const unsigned char* sfa = smem + s * kPairStageBytes + kPairStageA + kPairStageB;
           const unsigned char* sfb = sfa + kPairStageSfa;
-          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kPairStageSfb / 2, sf_buf_col(b));
+          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kPairStageSfb / 2, sf_buf_col(s));
           tmem_st_wait();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_remote(sf_ready_leader + 8u * (uint32_t)b);   // this CTA's stage + scales ready
+        if (lane == 0) mbar_arrive_remote(sf_ready_leader + 8u * (uint32_t)s);   // this CTA's stage + scales ready
       }
     }
   } else if (warp == kMmaWarp) {
@@ -189,8 +188,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         }
         tc_fence_after();
         for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-          const int s = it % STAGES, b = it % kSfBufs;
-          if (!mbar_wait_cluster(sf_ready + b, (it / kSfBufs) & 1u, kDevErrTimeoutScales)) {
+          const int s = it % STAGES;
+          // both CTAs' scale warps saw stage s full and put its scales in TMEM
+          if (!mbar_wait_cluster(sf_ready + s, (it / STAGES) & 1u, kDevErrTimeoutScales)) {
             ok = false;
             break;
           }
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
           const uint32_t sa = smem_u32(smem + s * kPairStageBytes);
           const uint32_t sb = sa + kPairStageA;
           if (kt < n_fp4_kt) {
-            const uint32_t sfa = tmem + sf_buf_col(b);
+            const uint32_t sfa = tmem + sf_buf_col(s);
             const uint32_t sfb = sfa + 4 * kGemmKBPerStage;
             const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
             for (int kb = 0; kb < kbs; ++kb) {
@@ -215,8 +215,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
               mma_bf16_pair(tmem, ad, bd, idesc_lr, 1u);
             }
           }
-          tc_commit_pair(empty + s, 0x3);     // stage s of both CTAs is free once these MMAs read it
-          tc_commit_pair(sf_free + b, 0x3);   // and so is scale buffer b of both CTAs
+          tc_commit_pair(empty + s, 0x3);     // stage s and its scale buffer, in both CTAs, are free
         }
         tc_commit_pair(acc_full, 0x3);        // both halves of the tile's accumulator are complete
       }
