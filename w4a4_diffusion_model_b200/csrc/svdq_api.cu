@@ -15,6 +15,7 @@
 #include "svdq_gemm_pair.cuh"
 #include "svdq_prepare.cuh"
 #include "svdq_quant.cuh"
+#include "svdq_quant_tma.cuh"
 #include "svdq_svd.cuh"
 
 namespace {
@@ -143,19 +144,122 @@ svdq_status make_scale_tmap(CUtensorMap* tm, const void* base, int64_t rows, int
 size_t scale_bytes(int64_t rows, int64_t K) { return (size_t)((rows + 127) / 128) * (size_t)(K / 64) * 512u; }
 
 // ---------------------------------------------------------------- launchers
+int sm_count() {
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  int n = 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
+  if (dev < 64) cached[dev] = n;
+  return n;
+}
+
+// Quantization: one CTA per BM rows (128 or 64) and K slice, one CTA per SM.
+// Every configuration covers ceil(M/128)*128 rows, so the padding rows of the
+// last scale atom get zero scales. With a low-rank branch the K slices of a
+// row block form a cluster (their partial T is summed through distributed
+// shared memory) and all clusters must be resident at once.
+template <int RANK, int BM, bool QUANT>
+struct QuantLaunch {
+  using L = svdq::QuantSmem<RANK, BM>;
+  static constexpr auto kern = svdq::quantize_tma_kernel<RANK, BM, QUANT>;
+
+  static svdq_status prepare() {   // once per device
+    static bool done[64];
+    int dev = 0;
+    SVDQ_CUDA(cudaGetDevice(&dev));
+    if (dev >= 64 || !done[dev]) {
+      SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
+      if (dev < 64) done[dev] = true;
+    }
+    return SVDQ_OK;
+  }
+
+  // Clusters of k CTAs that can be resident at once (cached per k).
+  static int max_clusters(int k) {
+    static int cache[4] = {-1, -1, -1, -1};
+    const int i = k == 2 ? 1 : k == 4 ? 2 : 3;
+    if (cache[i] < 0) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = k;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(k, 1, 1);
+      cfg.blockDim = dim3(L::kThreads, 1, 1);
+      cfg.dynamicSmemBytes = L::kBytes;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+      cudaGetLastError();
+      cache[i] = n;
+    }
+    return cache[i];
+  }
+
+  // Largest K split (8, 4, 2, 1) that keeps the grid in one wave; returns the
+  // CTA count, 0 when K is not a whole number of stages.
+  static int plan(const svdq_shape& s, int* ksplit) {
+    *ksplit = 1;
+    if (s.K % L::kCols) return 0;
+    const int rowblocks = (int)((s.M + 127) / 128) * (128 / BM);
+    const int nst = (int)(s.K / L::kCols);
+    for (int k = 8; k >= 2; k /= 2) {
+      if (nst % k || rowblocks * k > sm_count()) continue;
+      if (RANK > 0 && rowblocks > max_clusters(k)) continue;
+      *ksplit = k;
+      return rowblocks * k;
+    }
+    *ksplit = 1;
+    return rowblocks;
+  }
+
+  static svdq_status launch(const svdq_shape& s, int ksplit, const void* X, const float* inv, const void* L1p,
+                            void* Qx, void* Sx, void* T, cudaStream_t st) {
+    const int rowblocks = (int)((s.M + 127) / 128) * (128 / BM);
+    CUtensorMap tx, tl;
+    std::memset(&tl, 0, sizeof(tl));
+    svdq_status r;
+    if ((r = make_tmap(&tx, X, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.K, (uint64_t)s.M, 64, BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+    if (RANK > 0 && (r = make_tmap(&tl, L1p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.K, (uint64_t)RANK,
+                                   64, RANK, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ksplit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(rowblocks * ksplit, 1, 1);
+    cfg.blockDim = dim3(L::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::kBytes;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = (RANK > 0 && ksplit > 1) ? 1 : 0;
+    SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tx, tl, inv, static_cast<uint8_t*>(Qx), static_cast<uint8_t*>(Sx),
+                                 static_cast<__nv_bfloat16*>(T), (int)s.M, (int)s.K, ksplit));
+    return SVDQ_OK;
+  }
+};
+
+// 128-row CTAs unless 64-row CTAs put more of them in the one wave.
 template <int RANK, bool QUANT>
 svdq_status launch_quant_t(const svdq_shape& s, const void* X, const float* inv, const void* L1p, void* Qx, void* Sx,
                            void* T, cudaStream_t st) {
-  const int rows = QUANT ? (int)((s.M + 127) / 128 * 128) : (int)((s.M + 15) / 16 * 16);
-  const int grid = rows / svdq::kQuantRows;
-  const size_t smem = RANK > 0 ? (size_t)8 * svdq::kQuantRows * RANK * sizeof(float) : 0;
-  auto kern = svdq::quantize_act_kernel<RANK, QUANT>;
-  if (smem > 48 * 1024) SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-  kern<<<grid, svdq::kQuantThreads, smem, st>>>(
-      static_cast<const __nv_bfloat16*>(X), inv, static_cast<const __nv_bfloat16*>(L1p), static_cast<uint8_t*>(Qx),
-      static_cast<uint8_t*>(Sx), static_cast<__nv_bfloat16*>(T), (int)s.M, (int)s.K);
-  SVDQ_LAUNCHED("quantize_act_kernel");
-  return SVDQ_OK;
+  using Big = QuantLaunch<RANK, 128, QUANT>;
+  using Small = QuantLaunch<RANK, 64, QUANT>;
+  if (s.M == 0) return SVDQ_OK;
+  svdq_status r;
+  if ((r = Big::prepare()) != SVDQ_OK || (r = Small::prepare()) != SVDQ_OK) return r;
+  int kb = 1, ks = 1;
+  const int nb = Big::plan(s, &kb), ns = Small::plan(s, &ks);
+  if (ns > nb && ns <= sm_count()) return Small::launch(s, ks, X, inv, L1p, Qx, Sx, T, st);
+  return Big::launch(s, kb, X, inv, L1p, Qx, Sx, T, st);
 }
 
 template <bool QUANT>
@@ -171,17 +275,6 @@ svdq_status launch_quant(const svdq_shape& s, int rank, const void* X, const flo
     default:
       return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d", rank);
   }
-}
-
-int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 64 && cached[dev]) return cached[dev];
-  int n = 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-  if (dev < 64) cached[dev] = n;
-  return n;
 }
 
 constexpr int kGemmStages = 3;

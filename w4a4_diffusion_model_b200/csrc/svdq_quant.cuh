@@ -1,9 +1,9 @@
-// Activation-side kernels of the SVDQuant W4A4 layer:
-//   * quantize_act_kernel: smoothing, NVFP4 group quantization and (fused)
-//     the low-rank down-projection T = X L1' from one read of X
-//     (devpress.csdn.net SVDQuant walkthrough, eq. (1), eq. (5), Fig. 6);
+// Activation-side helpers of the SVDQuant W4A4 layer (the quantization kernel
+// itself is quantize_tma_kernel):
+//   * nvfp4_encode16: the NVFP4 group recipe (also used for the weights);
 //   * channel_amax_kernel: per-channel max|x| (handbook SmoothQuant section);
-//   * scales_native_to_canonical_kernel: inspection helper.
+//   * scales_native_to_canonical_kernel: inspection helper;
+//   * lowrank_up_rmw_kernel: the unfused up-projection.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -51,25 +51,6 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& code
   codes = make_uint2(w[0], w[1]);
 }
 
-// One 16-element chunk of a bf16 row: 2 x 16-byte loads.
-struct Chunk16 {
-  uint32_t w[8];
-};
-
-__device__ __forceinline__ Chunk16 load_chunk16(const __nv_bfloat16* p, bool ok) {
-  Chunk16 c;
-  if (ok) {
-    const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
-    const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
-    c.w[0] = a.x; c.w[1] = a.y; c.w[2] = a.z; c.w[3] = a.w;
-    c.w[4] = b.x; c.w[5] = b.y; c.w[6] = b.z; c.w[7] = b.w;
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) c.w[i] = 0u;
-  }
-  return c;
-}
-
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(
@@ -77,119 +58,6 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint3
       "{%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-constexpr int kQuantThreads = 256;   // 8 warps
-constexpr int kQuantRows = 16;       // rows per CTA (one m16 MMA tile)
-
-// Grid: one CTA per 16 rows of ceil(M/128)*128 rows (padding rows only write
-// zero scales so the native scale atoms are fully defined). Warp w walks the
-// 64-column slabs w, w+8, ...; thread (g = lane/4, t = lane%4) owns rows
-// m0+g and m0+g+8, columns [64 s + 16 t, +16) of slab s — one quantization
-// group per row. The down-projection reuses the same registers as mma.sync
-// A fragments: in k-step ks of a slab, the MMA's reduction index
-// {2t, 2t+1, 2t+8, 2t+9} maps to columns 64 s + 16 t + 4 ks + {0, 1, 2, 3}, and
-// the B fragment (L1p row n, same columns) is one 8-byte piece of L1p.
-// Partial T of the 8 warps is summed in shared memory in fixed warp order.
-template <int RANK, bool QUANT>
-__global__ void __launch_bounds__(kQuantThreads) quantize_act_kernel(
-    const __nv_bfloat16* __restrict__ X, const float* __restrict__ inv_lambda,
-    const __nv_bfloat16* __restrict__ L1p, uint8_t* __restrict__ Qx, uint8_t* __restrict__ Sx,
-    __nv_bfloat16* __restrict__ T, int M, int K) {
-  constexpr int NT = RANK / 8;
-  extern __shared__ float red[];   // [8][16][RANK]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, t = lane & 3;
-  const int m0 = blockIdx.x * kQuantRows;
-  const int rA = m0 + g, rB = m0 + g + 8;
-  const bool okA = rA < M, okB = rB < M;
-  const int nslab = K >> 6;
-  const size_t ldq = (size_t)K >> 1;
-
-  float acc[NT > 0 ? NT : 1][4];
-#pragma unroll
-  for (int i = 0; i < (NT > 0 ? NT : 1); ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-
-  if (m0 < M || QUANT) {
-#pragma unroll 1
-    for (int s = warp; s < nslab; s += 8) {
-      const int c = s * 64 + t * 16;
-      const Chunk16 xa = load_chunk16(X + (size_t)rA * K + c, okA);
-      const Chunk16 xb = load_chunk16(X + (size_t)rB * K + c, okB);
-
-      if constexpr (QUANT) {
-        float il[16];
-        const float4* ilp = reinterpret_cast<const float4*>(inv_lambda + c);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float4 f = __ldg(ilp + q);
-          il[4 * q] = f.x; il[4 * q + 1] = f.y; il[4 * q + 2] = f.z; il[4 * q + 3] = f.w;
-        }
-        uint32_t sbA, sbB;
-        uint2 qa, qb;
-        {
-          float v[16];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[2 * i] = __fmul_rn(bf16lo(xa.w[i]), il[2 * i]);
-            v[2 * i + 1] = __fmul_rn(bf16hi(xa.w[i]), il[2 * i + 1]);
-          }
-          nvfp4_encode16(v, qa, sbA);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            v[2 * i] = __fmul_rn(bf16lo(xb.w[i]), il[2 * i]);
-            v[2 * i + 1] = __fmul_rn(bf16hi(xb.w[i]), il[2 * i + 1]);
-          }
-          nvfp4_encode16(v, qb, sbB);
-        }
-        if (okA) *reinterpret_cast<uint2*>(Qx + (size_t)rA * ldq + (c >> 1)) = qa;
-        if (okB) *reinterpret_cast<uint2*>(Qx + (size_t)rB * ldq + (c >> 1)) = qb;
-        // The four scale bytes of one row and slab are adjacent in the native
-        // layout (group j = t): gather them to lane t == 0 and store one word.
-        const uint32_t a1 = __shfl_down_sync(0xFFFFFFFFu, sbA, 1), a2 = __shfl_down_sync(0xFFFFFFFFu, sbA, 2),
-                       a3 = __shfl_down_sync(0xFFFFFFFFu, sbA, 3);
-        const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sbB, 1), b2 = __shfl_down_sync(0xFFFFFFFFu, sbB, 2),
-                       b3 = __shfl_down_sync(0xFFFFFFFFu, sbB, 3);
-        if (t == 0) {
-          *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rA, s * 4, K)) =
-              sbA | (a1 << 8) | (a2 << 16) | (a3 << 24);
-          *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rB, s * 4, K)) =
-              sbB | (b1 << 8) | (b2 << 16) | (b3 << 24);
-        }
-      }
-
-      if constexpr (NT > 0) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          const Chunk16 l = load_chunk16(L1p + (size_t)(nt * 8 + g) * K + c, true);
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16_16816(acc[nt], xa.w[2 * ks], xb.w[2 * ks], xa.w[2 * ks + 1], xb.w[2 * ks + 1],
-                           l.w[2 * ks], l.w[2 * ks + 1]);
-        }
-      }
-    }
-  }
-
-  if constexpr (NT > 0) {
-    float* mine = red + (size_t)warp * kQuantRows * RANK;
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-      const int col = nt * 8 + 2 * t;
-      mine[g * RANK + col] = acc[nt][0];
-      mine[g * RANK + col + 1] = acc[nt][1];
-      mine[(g + 8) * RANK + col] = acc[nt][2];
-      mine[(g + 8) * RANK + col + 1] = acc[nt][3];
-    }
-    __syncthreads();
-    for (int e = threadIdx.x; e < kQuantRows * RANK; e += kQuantThreads) {
-      float s = 0.f;
-#pragma unroll
-      for (int w = 0; w < 8; ++w) s += red[w * kQuantRows * RANK + e];
-      const int row = m0 + e / RANK;
-      if (row < M) T[(size_t)row * RANK + (e % RANK)] = __float2bfloat16_rn(s);
-    }
-  }
 }
 
 // amax[j] = max_m |X[m][j]| over bf16 X [M][K]; amax must be zeroed first.

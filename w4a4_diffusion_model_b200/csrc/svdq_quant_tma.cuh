@@ -1,0 +1,320 @@
+// Activation quantization with the fused low-rank down-projection, fed by a
+// TMA ring (devpress.csdn.net SVDQuant walkthrough, eq. (1), eq. (5), Fig. 6:
+// the down-projection shares the quantizer's read of X).
+//
+// A CTA owns BM (128 or 64) rows of X and a slice of K. One producer thread
+// streams stages of 32 KB of X -- 16384/BM columns as 64-column x BM-row boxes
+// with 128B swizzle -- with the matching columns of L1p (64-column boxes of
+// RANK rows) and of inv_lambda, through a ring of stages (as many as fit in
+// shared memory, at most six).
+//
+// Quantization: 16 warps own 16 rows and one 64-column slab of every stage
+// each (with RG = BM/16 row groups, warp w takes rows 16 (w mod RG) + [0, 16)
+// and slab w / RG). Thread (g = lane/4, t = lane%4) quantizes rows g and g+8,
+// columns [16t, 16t+16) of the slab -- one quantization group per row.
+//
+// Down-projection: one thread issues tcgen05 kind::f16 MMAs on the same
+// shared-memory tiles (X box as A, L1p box as B, both K-major with 128B
+// swizzle), accumulating T = X L1p^T over the CTA's K slice in TMEM
+// (M = BM lanes, RANK fp32 columns). A stage is free once the quantizing warps
+// have read it and the MMAs that read it have completed. Four warps read the
+// accumulator back: with BM = 128 row r sits in TMEM lane r, with BM = 64 in
+// lane (r mod 16) + 32 (r div 16).
+//
+// With K split over a cluster of `ksplit` CTAs the partial sums of T are added
+// in cluster rank order through distributed shared memory.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp4.h>
+#include <cuda_fp8.h>
+
+#include "svdq_ptx.cuh"
+#include "svdq_quant.cuh"
+
+namespace svdq {
+
+constexpr int kQStageXBytes = 32768;       // X bytes per stage
+constexpr int kQMaxStages = 6;
+constexpr int kQSmemBudget = 227 * 1024 - 4096;   // leaves room for barriers, the 1 KB alignment and static tables
+
+template <int RANK, int BM>
+struct QuantSmem {
+  static_assert(BM == 128 || BM == 64, "rows per CTA");
+  static constexpr int kComputeWarps = 16;
+  static constexpr int kProducerWarp = kComputeWarps;
+  static constexpr int kMmaWarp = kComputeWarps + 1;
+  static constexpr int kThreads = 32 * (kComputeWarps + 2);
+  static constexpr int kRowGroups = BM / 16;
+  static constexpr int kCols = kQStageXBytes / (2 * BM);       // K columns per stage
+  static constexpr int kSlabs = kCols / 64;
+  static_assert(kRowGroups * kSlabs == kComputeWarps, "one slab per warp and stage");
+  static constexpr int kBoxBytes = 64 * BM * 2;
+  static constexpr int kL1Box = 64 * RANK * 2;
+  static constexpr int kL1 = kSlabs * kL1Box;
+  static constexpr int kInv = kCols * 4;
+  // 1 KB aligned stages: the 128B swizzle pattern repeats every 1024 bytes
+  static constexpr int kStage = (kQStageXBytes + kL1 + kInv + 1023) / 1024 * 1024;
+  static constexpr int kStages = kQSmemBudget / kStage < kQMaxStages ? kQSmemBudget / kStage : kQMaxStages;
+  static constexpr int kBarOffset = kStages * kStage;
+  static constexpr int kRedStride = RANK + 4;                  // fp32 partial T rows, padded against bank conflicts
+  static constexpr int kRed = BM * kRedStride * 4;             // reuses the ring
+  static constexpr uint32_t kTmemCols = RANK <= 32 ? 32 : RANK <= 64 ? 64 : 128;
+  static_assert(kRed <= kBarOffset, "partial sums must fit in the ring");
+  static_assert(kStages >= 2, "ring too shallow");
+  static constexpr int kBytes = kBarOffset + 256 + 1024;
+};
+
+// Byte offset of 16-byte chunk c of row r in a 128B-swizzled box (128-byte rows).
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
+
+// Two IEEE round-to-nearest fp32 products in one instruction.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// The NVFP4 recipe of nvfp4_encode16 for one group given as 8 packed bf16
+// pairs and its 16 inverse smoothing factors:
+//   v = fp32(x * inv_lambda); s = E4M3_rne_satfinite(fp32(max|v| / 6));
+//   q = E2M1_rne_satfinite(fp32(v * fp32(1/s))), all +0 when s is 0.
+// fp32(1/s) comes from `rcp_tbl`, indexed by the E4M3 byte of s.
+__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float* rcp_tbl,
+                                                  uint2& codes, uint32_t& sbyte) {
+  float2 v[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 l = *reinterpret_cast<const float4*>(il + 4 * q);
+    v[2 * q] = mul2_rn(make_float2(bf16lo(w[2 * q]), bf16hi(w[2 * q])), make_float2(l.x, l.y));
+    v[2 * q + 1] = mul2_rn(make_float2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1])), make_float2(l.z, l.w));
+  }
+  float m[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[i].x), fabsf(v[i].y));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
+  m[0] = fmaxf(m[0], m[2]);
+  m[1] = fmaxf(m[1], m[3]);
+  const float amax = fmaxf(m[0], m[1]);
+  const uint32_t b = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+  const float inv = rcp_tbl[b & 0x7Fu];
+  uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(mul2_rn(v[i], make_float2(inv, inv)), __NV_E2M1,
+                                                             cudaRoundNearest) & 0xFFu;
+    if (i < 4) lo |= byte << (8 * i);
+    else hi |= byte << (8 * (i - 4));
+  }
+  sbyte = b;
+  codes = b != 0u ? make_uint2(lo, hi) : make_uint2(0u, 0u);
+}
+
+template <int RANK, int BM, bool QUANT>
+__global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma_kernel(
+    const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
+    const float* __restrict__ inv_lambda, uint8_t* __restrict__ Qx, uint8_t* __restrict__ Sx,
+    __nv_bfloat16* __restrict__ T, int M, int K, int ksplit) {
+  if constexpr (!QUANT && RANK == 0) return;
+  using L = QuantSmem<RANK, BM>;
+  constexpr int RG = L::kRowGroups;
+  extern __shared__ __align__(1024) unsigned char qsmem_raw[];
+  __shared__ float rcp_tbl[128];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* empty = full + L::kStages;
+  uint64_t* acc_bar = empty + L::kStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_bar + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kslice = blockIdx.x % ksplit;            // == cluster rank when ksplit > 1
+  const int m0 = (blockIdx.x / ksplit) * BM;
+  const int nst = K / L::kCols / ksplit;
+  const int st0 = kslice * nst;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, (QUANT ? L::kComputeWarps : 0) + (RANK > 0 ? 1 : 0));
+    }
+    mbar_init(acc_bar, 1);
+    fence_mbar_init();
+  }
+  if (QUANT && threadIdx.x < 128) {   // fp32(1/s) for every E4M3 byte with the sign bit clear
+    const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)threadIdx.x, __NV_E4M3)));
+    rcp_tbl[threadIdx.x] = __frcp_rn(sv);
+  }
+  if (RANK > 0 && warp == L::kMmaWarp) {
+    tmem_alloc(tmem_slot, L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = RANK > 0 ? *tmem_slot : 0u;
+
+  if (warp == L::kProducerWarp) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tmap(&tm_x);
+      if (RANK > 0) prefetch_tmap(&tm_l1);
+      for (int j = 0; j < nst; ++j) {
+        const int s = j % L::kStages;
+        if (!mbar_wait(empty + s, ((j / L::kStages) & 1u) ^ 1u, kDevErrTimeoutEmpty)) break;
+        unsigned char* st = smem + s * L::kStage;
+        const int c0 = (st0 + j) * L::kCols;
+        mbar_arrive_expect_tx(full + s, (uint32_t)(kQStageXBytes + L::kL1 + (QUANT ? L::kInv : 0)));
+#pragma unroll
+        for (int b = 0; b < L::kSlabs; ++b) {
+          tma_load_2d(st + b * L::kBoxBytes, &tm_x, full + s, c0 + 64 * b, m0);
+          if (RANK > 0) tma_load_2d(st + kQStageXBytes + b * L::kL1Box, &tm_l1, full + s, c0 + 64 * b, 0);
+        }
+        if (QUANT) bulk_load(st + kQStageXBytes + L::kL1, inv_lambda + c0, (uint32_t)L::kInv, full + s);
+      }
+    }
+  } else if (warp == L::kMmaWarp) {
+    // ------------------------------------------------------------------ down-projection MMAs
+    if (RANK > 0 && lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(BM, RANK > 0 ? RANK : 16);
+      bool ok = true;
+      for (int j = 0; j < nst && ok; ++j) {
+        const int s = j % L::kStages;
+        if (!mbar_wait(full + s, (j / L::kStages) & 1u, kDevErrTimeoutFull)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t st = smem_u32(smem + s * L::kStage);
+#pragma unroll
+        for (int b = 0; b < L::kSlabs; ++b) {
+          const uint32_t sa = st + b * L::kBoxBytes, sb = st + kQStageXBytes + b * L::kL1Box;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {   // 16 bf16 (32 bytes) of K per MMA
+            const uint64_t ad = smem_desc(sa + 32 * k, 16, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(sb + 32 * k, 16, 1024, kSwizzle128B);
+            mma_bf16(tmem, ad, bd, idesc, (j | b | k) != 0 ? 1u : 0u);
+          }
+        }
+        tc_commit(empty + s);
+      }
+      tc_commit(acc_bar);
+    }
+  } else if (QUANT) {
+    // ------------------------------------------------------------------ quantizing warps
+    const int g = lane >> 2, t = lane & 3;
+    const int rl = (warp % RG) * 16 + g;             // local rows rl and rl + 8
+    const int h = warp / RG;                         // 64-column slab of every stage
+    const int rA = m0 + rl, rB = rA + 8;
+    const bool okA = rA < M, okB = rB < M;
+    const size_t ldq = (size_t)K >> 1;
+    for (int j = 0; j < nst; ++j) {
+      const int s = j % L::kStages;
+      if (!mbar_wait(full + s, (j / L::kStages) & 1u, kDevErrTimeoutFull)) break;
+      const unsigned char* st = smem + s * L::kStage;
+      const unsigned char* box = st + h * L::kBoxBytes;
+      uint32_t xa[8], xb[8];
+      {
+        const uint4 a0 = *reinterpret_cast<const uint4*>(box + sw128(rl, 2 * t));
+        const uint4 a1 = *reinterpret_cast<const uint4*>(box + sw128(rl, 2 * t + 1));
+        const uint4 b0 = *reinterpret_cast<const uint4*>(box + sw128(rl + 8, 2 * t));
+        const uint4 b1 = *reinterpret_cast<const uint4*>(box + sw128(rl + 8, 2 * t + 1));
+        xa[0] = a0.x; xa[1] = a0.y; xa[2] = a0.z; xa[3] = a0.w;
+        xa[4] = a1.x; xa[5] = a1.y; xa[6] = a1.z; xa[7] = a1.w;
+        xb[0] = b0.x; xb[1] = b0.y; xb[2] = b0.z; xb[3] = b0.w;
+        xb[4] = b1.x; xb[5] = b1.y; xb[6] = b1.z; xb[7] = b1.w;
+      }
+      const int c = (st0 + j) * L::kCols + 64 * h + 16 * t;   // first column of this thread's group
+      const float* il = reinterpret_cast<const float*>(st + kQStageXBytes + L::kL1) + 64 * h + 16 * t;
+      uint2 qa, qb;
+      uint32_t sbA, sbB;
+      encode_group_bf16(xa, il, rcp_tbl, qa, sbA);
+      encode_group_bf16(xb, il, rcp_tbl, qb, sbB);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty + s);         // the stage's shared memory is no longer read
+      if (okA) *reinterpret_cast<uint2*>(Qx + (size_t)rA * ldq + (c >> 1)) = qa;
+      if (okB) *reinterpret_cast<uint2*>(Qx + (size_t)rB * ldq + (c >> 1)) = qb;
+      // the four scale bytes of a row and slab are adjacent in the native layout
+      const uint32_t a1 = __shfl_down_sync(0xFFFFFFFFu, sbA, 1), a2 = __shfl_down_sync(0xFFFFFFFFu, sbA, 2),
+                     a3 = __shfl_down_sync(0xFFFFFFFFu, sbA, 3);
+      const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sbB, 1), b2 = __shfl_down_sync(0xFFFFFFFFu, sbB, 2),
+                     b3 = __shfl_down_sync(0xFFFFFFFFu, sbB, 3);
+      if (t == 0) {   // rows past M get zero scales: TMA zero-fills them
+        *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rA, c >> 4, K)) =
+            sbA | (a1 << 8) | (a2 << 16) | (a3 << 24);
+        *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rB, c >> 4, K)) =
+            sbB | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      }
+    }
+  }
+
+  if constexpr (RANK > 0) {
+    // ------------------------------------------------------------------ T from TMEM
+    __syncthreads();   // every role has left its loop: the ring is free once the MMAs are done
+    float* red = reinterpret_cast<float*>(smem);   // [BM rows][kRedStride], partial T of this K slice
+    if (warp < 4) {
+      // warp q reads TMEM lanes 32q..32q+31: rows 32q + lane (BM = 128) or 16q + lane, lane < 16 (BM = 64)
+      const bool live = BM == 128 || lane < 16;
+      const int r = BM == 128 ? 32 * warp + lane : 16 * warp + lane;
+      const bool acc_ok = mbar_wait(acc_bar, 0u, kDevErrTimeoutAccum);
+      tc_fence_after();
+#pragma unroll
+      for (int c = 0; c < RANK / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * warp) << 16) + 16u * c, v);
+        tmem_ld_wait();
+        if (!live || !acc_ok) continue;
+        if (ksplit == 1) {
+          if (m0 + r < M) {
+            uint32_t p[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+              p[i] = *reinterpret_cast<const uint32_t*>(&bb);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(T + (size_t)(m0 + r) * RANK + 16 * c);
+            dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
+            dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
+          }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(red + r * L::kRedStride + 16 * c);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == L::kMmaWarp) {
+      tc_fence_after();
+      tmem_dealloc(tmem, L::kTmemCols);
+    }
+    if (ksplit > 1) {
+      cluster_sync();
+      // CTA kslice finalises rows [kslice * BM / ksplit, ...), adding the slices in rank order
+      const int rows_per = BM / ksplit;
+      const int e0 = kslice * rows_per * RANK, e1 = e0 + rows_per * RANK;
+      const uint32_t red_addr = smem_u32(red);
+      for (int e = e0 + (int)threadIdx.x; e < e1; e += L::kThreads) {
+        const int row = e / RANK, col = e % RANK;
+        const uint32_t off = 4u * (uint32_t)(row * L::kRedStride + col);
+        float sum = 0.f;
+        for (int p = 0; p < ksplit; ++p) {
+          float x;
+          const uint32_t a = mapa_shared(red_addr + off, (uint32_t)p);
+          asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(a) : "memory");
+          sum += x;
+        }
+        if (m0 + row < M) T[(size_t)(m0 + row) * RANK + col] = __float2bfloat16_rn(sum);
+      }
+      cluster_sync();   // peers keep their partial sums until everyone has read them
+    }
+  }
+}
+
+}  // namespace svdq
