@@ -15,12 +15,14 @@ no data-path collective); the step time is the max over ranks, the value the
 FLOPs of all ranks over that time (weak scaling).
 
 Timing: W untimed warm-up steps; each timed step is bracketed by CUDA events
-on the launching stream, with a write of a 256 MiB buffer (larger than the
-126 MB L2) between steps so that every step starts with a cold L2.
+on the launching stream. Steps rotate over copies of X and of the prepared
+weights whose total exceeds twice the 126 MB L2, so every step reads its
+inputs from HBM (as a network whose layers each have their own weights would).
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -69,6 +71,19 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
+def weight_bytes(P) -> int:
+    return sum(t.numel() * t.element_size() for t in (P.Qr, P.Sr, P.L1p, P.L2t, P.lam, P.inv_lam) if t is not None)
+
+
+def clone_weights(P):
+    """A copy of prepared weights in fresh device buffers."""
+    return dataclasses.replace(P, **{f: (getattr(P, f).clone() if getattr(P, f) is not None else None)
+                                     for f in ("Qr", "Sr", "L1p", "L2t", "lam", "inv_lam")})
+
+
 def quantize_bytes(w: synth.Workload) -> int:
     """Algorithmic HBM bytes of one quantize launch: read X, inv_lambda, L1p;
     write codes, scales (rows padded to 128) and T."""
@@ -82,13 +97,14 @@ def gemm_flops(w: synth.Workload) -> int:
 
 
 GEMM_SOURCES = ("svdq_gemm.cuh", "svdq_gemm_pair.cuh", "svdq_gemm_common.cuh", "svdq_ptx.cuh")
+QUANT_SOURCES = ("svdq_quant_tma.cuh", "svdq_quant.cuh", "svdq_ptx.cuh")
 
 
-def kernel_source_hash() -> str:
-    """Hash of the GEMM kernel sources: ties a committed ncu traffic figure to
-    the kernel version it was measured on."""
+def kernel_source_hash(sources=GEMM_SOURCES) -> str:
+    """Hash of a kernel's sources: ties a committed ncu traffic figure to the
+    kernel version it was measured on."""
     h = hashlib.sha256()
-    for name in GEMM_SOURCES:
+    for name in sources:
         with open(os.path.join(ROOT, "w4a4_diffusion_model_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -98,13 +114,13 @@ def gemm_kernel_name(w: synth.Workload) -> str:
     return "svdq_gemm_pair_kernel" if w.N % 256 == 0 else "svdq_gemm_kernel"
 
 
-def profiled_traffic(workload: str):
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current kernel source for this workload; else None."""
-    p = os.path.join(ROOT, "profiles", f"svdq_gemm_{workload}.md")
+def profiled_traffic(summary: str, sources):
+    """DRAM bytes per launch from a committed ncu summary under profiles/, if
+    it was taken on the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", summary)
     if not os.path.exists(p):
         return None
-    src_hash = kernel_source_hash()
+    src_hash = kernel_source_hash(sources)
     with open(p) as f:
         for line in f:
             if line.startswith("traffic_bytes_per_launch:"):
@@ -334,27 +350,39 @@ def run_ours(args):
     Sx = torch.empty(sx_b, dtype=torch.uint8, device=dev)
     T = torch.empty(w.M, w.rank, dtype=torch.bfloat16, device=dev) if w.rank else None
     Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(P_=P, variant=S.SVDQ_FUSED, ev=None):
+    # L2: every step reads its own copy of X and of the prepared weights; the
+    # copies together exceed twice the L2, so each step starts from HBM.
+    set_bytes = X.numel() * 2 + weight_bytes(P)
+    n_sets = max(2, min(16, -(-2 * L2_BYTES // set_bytes)))
+    sets = [(X, P, P0)] + [(X.clone(), clone_weights(P), clone_weights(P0)) for _ in range(n_sets - 1)]
+    l2_note = f"rotating {n_sets} input sets (X + prepared weights, {set_bytes / 1e6:.1f} MB each) > 2x L2"
+
+    def step(i=0, rank0=False, variant=S.SVDQ_FUSED, ev=None):
+        X_, P_, P0_ = sets[i % n_sets]
+        if rank0:
+            P_ = P0_
+        r = P_.shape.rank
         if ev is not None:
             ev[0].record(stream)
-        S.svdq_quantize_act(X, P_.inv_lam, P_.L1p, P_.shape.rank, w.N, variant, out=(Qx, Sx, T if P_.shape.rank else None))
+        S.svdq_quantize_act(X_, P_.inv_lam, P_.L1p, r, w.N, variant, out=(Qx, Sx, T if r else None))
         if ev is not None:
             ev[1].record(stream)
-        S.svdq_linear(Qx, Sx, T if P_.shape.rank else None, P_, variant, out=Y)
+        S.svdq_linear(Qx, Sx, T if r else None, P_, variant, out=Y)
         if ev is not None:
             ev[2].record(stream)
 
     def timed(n, fn, warm=3):
-        for _ in range(warm):      # untimed: first-call setup (library handles, heuristics) stays out
-            flush.zero_()
-            fn([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+        """Per-step CUDA events around the two kernels. A GPU-side delay first
+        lets the host queue the steps ahead of the device."""
+        for i in range(warm):      # untimed: first-call setup (library handles, heuristics) stays out
+            fn(i, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
         for i in range(n):
-            flush.zero_()
-            fn(evs[i])
+            fn(i, evs[i])
         torch.cuda.synchronize()
         k1 = [evs[i][0].elapsed_time(evs[i][1]) for i in range(n)]
         k2 = [evs[i][1].elapsed_time(evs[i][2]) for i in range(n)]
@@ -365,17 +393,17 @@ def run_ours(args):
         t_load = time.time()
         t_end = t_load + 1.5
         while time.time() < t_end and (clk.n_samples() < 2 or time.time() < t_load + 0.6):
-            for _ in range(20):
-                step()
+            for i in range(20):
+                step(i)
             torch.cuda.synchronize()
-        for _ in range(args.warmup):
-            step()
+        for i in range(args.warmup):
+            step(i)
         S.svdq_check()
         if world > 1:
             torch.distributed.barrier()
         torch.cuda.synchronize()
         t0 = time.time()
-        k1, k2 = timed(args.steps, lambda ev: step(ev=ev), warm=0)
+        k1, k2 = timed(args.steps, lambda i, ev: step(i, ev=ev), warm=0)
         torch.cuda.synchronize()
         t1 = time.time()
         if world > 1:
@@ -395,7 +423,7 @@ def run_ours(args):
     k2_ms = statistics.mean(k2)
     k1_ms = statistics.mean(k1)
     achieved = gemm_flops(w) / (k2_ms * 1e-3) / 1e12
-    traffic = profiled_traffic(w.name)
+    traffic = profiled_traffic(f"svdq_gemm_{w.name}.md", GEMM_SOURCES)
     roofline = {"bound": "tensor", "kernel": gemm_kernel_name(w), "achieved": round(achieved, 2),
                 "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                 "traffic": traffic,
@@ -404,8 +432,9 @@ def run_ours(args):
                              f"vs 9000 TFLOP/s datasheet: {achieved / 9000:.4f}; "
                              f"vs {FP4_PER_BF16:g} x burst bf16: {achieved / (FP4_PER_BF16 * peaks['bf16_tflops']):.4f}"}
     q_gbs = quantize_bytes(w) / (k1_ms * 1e-3) / 1e9
-    roofline_q = {"bound": "hbm", "kernel": "quantize_act_kernel", "achieved": round(q_gbs, 1),
+    roofline_q = {"bound": "hbm", "kernel": "quantize_tma_kernel", "achieved": round(q_gbs, 1),
                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / peaks["hbm_gbs"], 4),
+                  "traffic": profiled_traffic(f"quantize_tma_{w.name}.md", QUANT_SOURCES),
                   "algorithmic_bytes": quantize_bytes(w)}
 
     extras = {}
@@ -414,16 +443,20 @@ def run_ours(args):
     if not args.no_extras:
         n_x = max(5, args.steps // 2)
         # unfused variant (same arithmetic, separate passes)
-        k1u, k2u = timed(n_x, lambda ev: step(variant=S.SVDQ_UNFUSED, ev=ev))
+        k1u, k2u = timed(n_x, lambda i, ev: step(i, variant=S.SVDQ_UNFUSED, ev=ev))
         # no low-rank branch (rank 0) on the same shape
         if w.rank:
-            k1z, k2z = timed(n_x, lambda ev: step(P_=P0, ev=ev))
+            k1z, k2z = timed(n_x, lambda i, ev: step(i, rank0=True, ev=ev))
         else:
             k1z, k2z = k1, k2
-        # bf16 cuBLAS X W^T through torch
-        def cublas(ev):
+        # bf16 cuBLAS X W^T through torch, rotating (X, W) copies the same way
+        n_c = max(2, min(8, -(-2 * L2_BYTES // (X.numel() * 2 + W.numel() * 2))))
+        cub_sets = [(X, W)] + [(X.clone(), W.clone()) for _ in range(n_c - 1)]
+
+        def cublas(i, ev):
+            Xc, Wc = cub_sets[i % n_c]
             ev[0].record(stream)
-            torch.nn.functional.linear(X, W)
+            torch.nn.functional.linear(Xc, Wc)
             ev[1].record(stream)
             ev[2].record(stream)
         kc, _ = timed(n_x, cublas)
@@ -444,7 +477,7 @@ def run_ours(args):
         X_host = X_cpu.pin_memory()
         Y_host = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
 
-        def e2e_step(ev):
+        def e2e_step(i, ev):
             ev[0].record(stream)
             X.copy_(X_host, non_blocking=True)
             S.svdq_quantize_act(X, P.inv_lam, P.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
@@ -473,10 +506,11 @@ def run_ours(args):
             "data": "synthetic",
             "config": {"workload": w.name, "M_per_gpu": w.M, "K": w.K, "N": w.N, "rank": w.rank, "alpha": w.alpha,
                        "global_tokens": w.M * world, "parallelism": f"token-parallel x{world} (weights replicated)",
-                       "l2": "flushed between steps (256 MiB write)"},
+                       "l2": l2_note},
             "roofline": roofline, "roofline_quantize": roofline_q,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 2 * args.steps, "clocks": clocks,
-            "extras": extras, "kernel_src": kernel_source_hash(),
+            "extras": extras,
+            "kernel_src": {"gemm": kernel_source_hash(GEMM_SOURCES), "quantize": kernel_source_hash(QUANT_SOURCES)},
         }
         print(json.dumps(line), flush=True)
         if args.extra_json:
