@@ -49,7 +49,24 @@ def test_size_queries():
     assert qx == 130 * 192 and sx == 2 * 6 * 512 and t == 0
     qr, sr, l1, l2, ws = S.svdq_weight_sizes(S.LayerShape(0, 12288, 3072, 32))
     assert qr == 3072 * 6144 and sr == 24 * 192 * 512 and l1 == 32 * 12288 * 2 and l2 == 3072 * 32 * 2
-    assert ws >= 0
+    assert ws > 0
+    *_, ws0 = S.svdq_weight_sizes(S.LayerShape(0, 12288, 3072, 0))
+    assert ws0 == 0                                   # no branch, no SVD
+    *_, ws128 = S.svdq_weight_sizes(S.LayerShape(0, 3072, 3072, 128))
+    assert ws128 > ws
+
+
+def test_prepare_without_factors_needs_the_workspace(lib):
+    """The device SVD runs in the caller's workspace: a missing or short one is
+    refused before any device work (rank 0 needs none)."""
+    sh = S.Shape(0, 512, 256, 16)
+    good = ctypes.c_void_p(1 << 20)
+    ws = ctypes.c_size_t()
+    assert lib.svdq_weight_sizes(sh, None, None, None, None, ctypes.byref(ws)) == 0
+    args = (good, good, ctypes.c_float(0.5), 0, good, good, good, good, good, good)
+    assert lib.svdq_prepare_weights(sh, *args, None, 0, None) == 4
+    assert lib.svdq_prepare_weights(sh, *args, good, ws.value - 256, None) == 4
+    assert b"workspace" in lib.svdq_last_error()
 
 
 @pytest.mark.parametrize("M,K,N,r", [(-1, 128, 128, 0), (1, 100, 128, 0), (1, 128, 100, 0), (1, 128, 128, 8),

@@ -22,13 +22,6 @@ namespace {
 
 thread_local char g_last_error[512] = "";
 
-void set_error(const char* fmt, ...) {
-  va_list ap;
-  va_start(ap, fmt);
-  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
-  va_end(ap);
-}
-
 svdq_status fail(svdq_status st, const char* fmt, ...) {
   va_list ap;
   va_start(ap, fmt);
@@ -432,6 +425,93 @@ svdq_status launch_up_rmw(const svdq_shape& s, int rank, const void* T, const vo
   }
 }
 
+// Randomized top-rank SVD of W_hat = diag(lambda) W_lin^T inside the caller's
+// workspace (plan and kernels in svdq_svd.cuh); writes L1p [r][K] and L2t [N][r].
+svdq_status launch_svd(const svdq_shape& s, const void* W, const float* lam, void* L1p, void* L2t, void* workspace,
+                       cudaStream_t st) {
+  using namespace svdq;
+  const SvdPlan p = svd_plan(s.K, s.N, s.rank);
+  const int K = (int)s.K, N = (int)s.N, l = p.l, r = s.rank;
+  char* ws = static_cast<char*>(workspace);
+  float* Y = reinterpret_cast<float*>(ws + p.off_ya);
+  float* Yalt = reinterpret_cast<float*>(ws + p.off_yb);
+  float* Z = reinterpret_cast<float*>(ws + p.off_za);
+  float* Zalt = reinterpret_cast<float*>(ws + p.off_zb);
+  float* part = reinterpret_cast<float*>(ws + p.off_part);
+  float* G = reinterpret_cast<float*>(ws + p.off_g);
+  float* V = reinterpret_cast<float*>(ws + p.off_v);
+  float* D = reinterpret_cast<float*>(ws + p.off_d);
+  float* T = reinterpret_cast<float*>(ws + p.off_t);
+  float* T2 = reinterpret_cast<float*>(ws + p.off_t2);
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
+  {
+    static bool done[64];
+    int dev = 0;
+    SVDQ_CUDA(cudaGetDevice(&dev));
+    if (dev >= 64 || !done[dev]) {
+      const int big = (int)jacobi_smem_bytes(kSvdMaxL), ab = (int)apply_smem_bytes(kSvdMaxL, kSvdMaxL);
+      SVDQ_CUDA(cudaFuncSetAttribute(svd_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
+      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
+      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyL1p>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
+      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyL2t>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
+      if (dev < 64) done[dev] = true;
+    }
+  }
+  auto grid_for = [](size_t n) { return (unsigned)((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048); };
+  auto eig_of_gram = [&](const float* buf, int rows, int parts) -> svdq_status {
+    svd_gram_kernel<<<parts, 256, 0, st>>>(buf, part, rows, l, parts);
+    SVDQ_LAUNCHED("svd_gram_kernel");
+    svd_reduce_kernel<<<grid_for((size_t)l * l), 256, 0, st>>>(part, nullptr, G, l, l, parts);
+    SVDQ_LAUNCHED("svd_reduce_kernel");
+    svd_jacobi_kernel<<<1, kJacobiThreads, jacobi_smem_bytes(l), st>>>(G, V, D, l);
+    SVDQ_LAUNCHED("svd_jacobi_kernel");
+    return SVDQ_OK;
+  };
+  auto svqb = [&](float*& buf, float*& alt, int rows, int parts) -> svdq_status {
+    for (int pass = 0; pass < 2; ++pass) {
+      svdq_status e = eig_of_gram(buf, rows, parts);
+      if (e != SVDQ_OK) return e;
+      svd_transform_kernel<<<1, 256, 0, st>>>(V, D, T, nullptr, l, l, 0);
+      SVDQ_LAUNCHED("svd_transform_kernel");
+      svd_apply_kernel<kApplyF32><<<rows / kSvdTile, 256, apply_smem_bytes(l, l), st>>>(buf, T, nullptr, alt,
+                                                                                        nullptr, rows, l, l);
+      SVDQ_LAUNCHED("svd_apply_kernel");
+      float* t = buf;
+      buf = alt;
+      alt = t;
+    }
+    return SVDQ_OK;
+  };
+  auto prod = [&](bool trans, const float* in, float* out) -> svdq_status {
+    const int rows = trans ? N : K, split = trans ? p.split_at : p.split_a;
+    const dim3 grid(rows / kSvdTile, split);
+    if (trans) svd_skinny_kernel<true><<<grid, 256, 0, st>>>(Wb, lam, in, part, N, K, l, split);
+    else svd_skinny_kernel<false><<<grid, 256, 0, st>>>(Wb, lam, in, part, N, K, l, split);
+    SVDQ_LAUNCHED("svd_skinny_kernel");
+    svd_reduce_kernel<<<grid_for((size_t)rows * l), 256, 0, st>>>(part, trans ? nullptr : lam, out, rows, l, split);
+    SVDQ_LAUNCHED("svd_reduce_kernel");
+    return SVDQ_OK;
+  };
+  svdq_status e;
+  svd_gaussian_kernel<<<grid_for((size_t)N * l), 256, 0, st>>>(Z, (size_t)N * l, kSvdSeed);
+  SVDQ_LAUNCHED("svd_gaussian_kernel");
+  if ((e = prod(false, Z, Y)) != SVDQ_OK || (e = svqb(Y, Yalt, K, p.parts_y)) != SVDQ_OK) return e;
+  for (int it = 0; it < kSvdPowerIters; ++it) {
+    if ((e = prod(true, Y, Z)) != SVDQ_OK || (e = svqb(Z, Zalt, N, p.parts_z)) != SVDQ_OK) return e;
+    if ((e = prod(false, Z, Y)) != SVDQ_OK || (e = svqb(Y, Yalt, K, p.parts_y)) != SVDQ_OK) return e;
+  }
+  if ((e = prod(true, Y, Z)) != SVDQ_OK || (e = eig_of_gram(Z, N, p.parts_z)) != SVDQ_OK) return e;
+  svd_transform_kernel<<<1, 256, 0, st>>>(V, D, T, T2, l, r, 1);
+  SVDQ_LAUNCHED("svd_transform_kernel");
+  svd_apply_kernel<kApplyL1p><<<K / kSvdTile, 256, apply_smem_bytes(l, r), st>>>(
+      Y, T, lam, nullptr, static_cast<__nv_bfloat16*>(L1p), K, l, r);
+  SVDQ_LAUNCHED("svd_apply_kernel");
+  svd_apply_kernel<kApplyL2t><<<N / kSvdTile, 256, apply_smem_bytes(l, r), st>>>(
+      Z, T2, nullptr, nullptr, static_cast<__nv_bfloat16*>(L2t), N, l, r);
+  SVDQ_LAUNCHED("svd_apply_kernel");
+  return SVDQ_OK;
+}
+
 svdq_status launch_channel_amax(int64_t rows, int64_t K, const void* X, float* amax, cudaStream_t st) {
   SVDQ_CUDA(cudaMemsetAsync(amax, 0, (size_t)K * sizeof(float), st));
   if (rows == 0) return SVDQ_OK;
@@ -531,10 +611,7 @@ svdq_status svdq_prepare_weights(svdq_shape s, const void* W, const float* act_a
                                                                               inv_lambda, (int)s.K);
   SVDQ_LAUNCHED("smoothing_lambda_kernel");
   if (s.rank > 0 && !given) {
-    if ((r = svdq::svd_lowrank_factors(s.K, s.N, s.rank, static_cast<const __nv_bfloat16*>(W), lambda,
-                                       static_cast<__nv_bfloat16*>(L1p), static_cast<__nv_bfloat16*>(L2t), workspace,
-                                       st, &set_error)) != SVDQ_OK)
-      return r;
+    if ((r = launch_svd(s, W, lambda, L1p, L2t, workspace, st)) != SVDQ_OK) return r;
   }
   const long long n_threads = s.N * (s.K / 16);
   svdq::residual_quantize_kernel<<<(unsigned)((n_threads + 127) / 128), 128, 0, st>>>(
