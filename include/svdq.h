@@ -120,8 +120,10 @@ SVDQ_API svdq_status svdq_channel_amax(int64_t M, int64_t K, const void* X, floa
  *   2. W_hat = diag(lambda) W_lin^T and its top-rank SVD split W_hat ~= L1 L2 with
  *      the singular values in L1 (walkthrough: SVD paragraph after eq. (8);
  *      handbook SVDQuant section). Without SVDQ_PREPARE_GIVEN_FACTORS the library
- *      computes it (randomized subspace iteration in fp64 on the device) and
- *      writes L1p and L2t; with it, L1p and L2t are read as given;
+ *      computes it on the device (randomized subspace iteration in fp32,
+ *      deterministic: a fixed seed and fixed reduction orders) and writes
+ *      L1p = bf16(L1 / lambda)^T [rank][K] and L2t = bf16(L2)^T [N][rank]; with
+ *      the flag, L1p and L2t are read as given;
  *   3. residual R = fp32(W_hat - sum_k (lambda * L1p[k]) L2t[:,k]) in fp64, in
  *      increasing k, no fused multiply-add (eq. (5));
  *   4. NVFP4 encoding of R grouped along K: codes Qr [N][K/2], native scales Sr.
