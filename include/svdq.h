@@ -136,6 +136,32 @@ SVDQ_API svdq_status svdq_prepare_weights(svdq_shape shape, const void* W_lin, c
                                  float* lambda, float* inv_lambda, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/* Size of the library's own device scratch used by svdq_prepare_weights_static. */
+#define SVDQ_STATIC_SCRATCH_BYTES ((size_t)32 << 20)
+
+/* svdq_prepare_weights without a workspace argument and without any
+ * allocation: the device SVD runs in one fixed scratch array of
+ * SVDQ_STATIC_SCRATCH_BYTES (32 MiB) that is part of the library's device
+ * image. The paper has no counterpart: this is a deployment convenience for
+ * callers that cannot hand out workspace memory. Same arguments, flags,
+ * arithmetic and outputs as svdq_prepare_weights (bit-identical results).
+ *   Limit.  Shapes whose SVD workspace (svdq_weight_sizes' workspace_bytes)
+ *     exceeds SVDQ_STATIC_SCRATCH_BYTES are refused with
+ *     SVDQ_ERR_BUFFER_TOO_SMALL and a message naming both sizes; use
+ *     svdq_prepare_weights with a caller workspace for those. The FLUX
+ *     projections at rank 32 need about 14 MB.
+ *   Set-up.  The first call on a device looks up the scratch's device address
+ *     (and sets kernel attributes) with that device current; make that first
+ *     call before capturing a stream into a CUDA graph.
+ *   Zero.  Nothing in the scratch needs to start at zero: every byte a call
+ *     reads was written earlier in the same call.
+ *   Concurrency.  There is one scratch per device and process. Calls whose
+ *     work overlaps on the device (other streams, other host threads) race on
+ *     it and corrupt each other's factors; serialize them. */
+SVDQ_API svdq_status svdq_prepare_weights_static(svdq_shape shape, const void* W_lin, const float* act_amax,
+                                                 float alpha, unsigned int flags, void* L1p, void* L2t, void* Qr,
+                                                 void* Sr, float* lambda, float* inv_lambda, void* stream);
+
 /* Per-call activation quantization with the low-rank down-projection.
  * X bf16 [M][K]; inv_lambda fp32 [K]; L1p bf16 [rank][K].
  * Writes Qx codes [M][K/2], Sx native scales, T bf16 [M][rank]:

@@ -18,6 +18,10 @@
 #include "svdq_quant_tma.cuh"
 #include "svdq_svd.cuh"
 
+// Device scratch of svdq_prepare_weights_static: the SVD workspace for callers
+// that provide none. Every byte a call reads is written earlier in that call.
+static __device__ __align__(256) unsigned char g_prepare_scratch[SVDQ_STATIC_SCRATCH_BYTES];
+
 namespace {
 
 thread_local char g_last_error[512] = "";
@@ -620,6 +624,43 @@ svdq_status svdq_prepare_weights(svdq_shape s, const void* W, const float* act_a
       (int)s.K, (int)s.rank);
   SVDQ_LAUNCHED("residual_quantize_kernel");
   return SVDQ_OK;
+}
+
+svdq_status svdq_prepare_weights_static(svdq_shape s, const void* W, const float* act_amax, float alpha,
+                                        unsigned int flags, void* L1p, void* L2t, void* Qr, void* Sr, float* lambda,
+                                        float* inv_lambda, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (flags & ~(unsigned)SVDQ_PREPARE_GIVEN_FACTORS) return fail(SVDQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  const bool given = (flags & SVDQ_PREPARE_GIVEN_FACTORS) != 0;
+  const size_t need = (given || s.rank == 0) ? 0 : svdq::svd_workspace_bytes(s.K, s.N, s.rank);
+  if (need > SVDQ_STATIC_SCRATCH_BYTES)
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL,
+                "shape K=%lld N=%lld rank=%d needs %zu bytes of SVD scratch, the static scratch holds %zu: "
+                "use svdq_prepare_weights with a caller workspace",
+                (long long)s.K, (long long)s.N, (int)s.rank, need, (size_t)SVDQ_STATIC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (need > 0) {
+    if ((r = check_device()) != SVDQ_OK) return r;
+    // device address of the scratch, looked up once per device with that device current
+    static std::mutex mu;
+    static void* addr[64];
+    int dev = 0;
+    SVDQ_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return fail(SVDQ_ERR_INTERNAL, "device ordinal %d out of range", dev);
+    std::lock_guard<std::mutex> lk(mu);
+    if (!addr[dev]) {
+      void* p = nullptr;
+      const cudaError_t e = cudaGetSymbolAddress(&p, g_prepare_scratch);
+      if (e != cudaSuccess || !p)
+        return fail(SVDQ_ERR_CUDA, "cudaGetSymbolAddress(static scratch): %s", cudaGetErrorString(e));
+      addr[dev] = p;
+    }
+    scratch = addr[dev];
+  }
+  return svdq_prepare_weights(s, W, act_amax, alpha, flags, L1p, L2t, Qr, Sr, lambda, inv_lambda, scratch, need,
+                              stream);
 }
 
 svdq_status svdq_quantize_act(svdq_shape s, const void* X, const float* inv_lambda, const void* L1p, void* Qx,

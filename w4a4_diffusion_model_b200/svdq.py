@@ -29,8 +29,8 @@ STATUS = {
 # Every symbol the header declares, with its ctypes signature.
 EXPORTS = [
     "svdq_status_string", "svdq_last_error", "svdq_version", "svdq_act_sizes", "svdq_weight_sizes",
-    "svdq_channel_amax", "svdq_prepare_weights", "svdq_quantize_act", "svdq_linear",
-    "svdq_scales_to_canonical", "svdq_check",
+    "svdq_channel_amax", "svdq_prepare_weights", "svdq_prepare_weights_static", "svdq_quantize_act",
+    "svdq_linear", "svdq_scales_to_canonical", "svdq_check",
 ]
 
 
@@ -67,6 +67,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_prepare_weights.argtypes = [Shape, vp, vp, ctypes.c_float, ctypes.c_uint, vp, vp, vp, vp, vp, vp,
                                          vp, sz, vp]
     lib.svdq_prepare_weights.restype = st
+    lib.svdq_prepare_weights_static.argtypes = [Shape, vp, vp, ctypes.c_float, ctypes.c_uint, vp, vp, vp, vp, vp,
+                                                vp, vp]
+    lib.svdq_prepare_weights_static.restype = st
     lib.svdq_quantize_act.argtypes = [Shape, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
     lib.svdq_quantize_act.restype = st
     lib.svdq_linear.argtypes = [Shape, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
