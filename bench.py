@@ -367,20 +367,27 @@ def run_ours(args):
         if ev is not None:
             ev[2].record(stream)
 
-    def timed(n, fn, warm=3):
-        """Per-step CUDA events around the two kernels. A GPU-side delay first
-        lets the host queue the steps ahead of the device."""
+    def timed(n, fn, warm=3, nlegs=0):
+        """Per-step CUDA events around the two kernels (for each of `nlegs`
+        interleaved legs when nlegs > 0). A GPU-side delay first lets the host
+        queue the steps ahead of the device."""
+        def events():
+            mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            return [mk() for _ in range(nlegs)] if nlegs else mk()
         for i in range(warm):      # untimed: first-call setup (library handles, heuristics) stays out
-            fn(i, [torch.cuda.Event(enable_timing=True) for _ in range(3)])
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+            fn(i, events())
+        evs = [events() for _ in range(n)]
         torch.cuda.synchronize()
         torch.cuda._sleep(2_000_000)
         for i in range(n):
             fn(i, evs[i])
         torch.cuda.synchronize()
-        k1 = [evs[i][0].elapsed_time(evs[i][1]) for i in range(n)]
-        k2 = [evs[i][1].elapsed_time(evs[i][2]) for i in range(n)]
-        return k1, k2
+
+        def split(ev_list):
+            return ([e[0].elapsed_time(e[1]) for e in ev_list], [e[1].elapsed_time(e[2]) for e in ev_list])
+        if nlegs:
+            return [split([evs[i][leg] for i in range(n)]) for leg in range(nlegs)]
+        return split(evs)
 
     with ClockSampler(smi_index(local)) as clk:
         # spin-up: keep the GPU loaded until the sampler reports, then warm up
@@ -436,13 +443,14 @@ def run_ours(args):
     cpu = None
     if not args.no_extras:
         n_x = max(5, args.steps // 2)
-        # unfused variant (same arithmetic, separate passes)
-        k1u, k2u = timed(n_x, lambda i, ev: step(i, variant=S.SVDQ_UNFUSED, ev=ev))
-        # no low-rank branch (rank 0) on the same shape
+        # fused, unfused (same arithmetic, separate passes) and no branch (rank 0)
+        # interleaved step by step, so that the comparison sees the same clocks
+        legs = [lambda i, ev: step(i, ev=ev), lambda i, ev: step(i, variant=S.SVDQ_UNFUSED, ev=ev)]
         if w.rank:
-            k1z, k2z = timed(n_x, lambda i, ev: step(i, rank0=True, ev=ev))
-        else:
-            k1z, k2z = k1, k2
+            legs.append(lambda i, ev: step(i, rank0=True, ev=ev))
+        res = timed(n_x, lambda i, ev: [f(i, e) for f, e in zip(legs, ev)], nlegs=len(legs))
+        (k1f, k2f), (k1u, k2u) = res[0], res[1]
+        k1z, k2z = res[2] if w.rank else res[0]
         # bf16 cuBLAS X W^T through torch, rotating (X, W) copies the same way
         n_c = max(2, min(8, -(-2 * L2_BYTES // (X.numel() * 2 + W.numel() * 2))))
         cub_sets = [(X, W)] + [(X.clone(), W.clone()) for _ in range(n_c - 1)]
@@ -455,6 +463,7 @@ def run_ours(args):
             ev[2].record(stream)
         kc, _ = timed(n_x, cublas)
         lay = statistics.mean(step_ms)
+        lay_f = statistics.mean(a + b for a, b in zip(k1f, k2f))
         extras = {
             "prepare_ms_offline": round(prepare_ms, 3),
             "quantize_ms": round(k1_ms, 4), "gemm_ms": round(k2_ms, 4), "layer_ms": round(lay, 4),
@@ -464,8 +473,10 @@ def run_ours(args):
             "bf16_cublas_ms": round(statistics.mean(kc), 4),
             "bf16_cublas_tflops": round(2 * w.M * w.N * w.K / (statistics.mean(kc) * 1e-3) / 1e12, 1),
         }
-        extras["lowrank_overhead_layer"] = round(lay / extras["rank0_layer_ms"] - 1, 4)
-        extras["lowrank_overhead_gemm"] = round(k2_ms / extras["rank0_gemm_ms"] - 1, 4)
+        extras["interleaved_fused_layer_ms"] = round(lay_f, 4)
+        extras["interleaved_fused_gemm_ms"] = round(statistics.mean(k2f), 4)
+        extras["lowrank_overhead_layer"] = round(lay_f / extras["rank0_layer_ms"] - 1, 4)
+        extras["lowrank_overhead_gemm"] = round(statistics.mean(k2f) / extras["rank0_gemm_ms"] - 1, 4)
         extras["unfused_overhead_layer"] = round(extras["unfused_layer_ms"] / extras["rank0_layer_ms"] - 1, 4)
 
         # end to end through the public API with host buffers: pinned X in, Y out
