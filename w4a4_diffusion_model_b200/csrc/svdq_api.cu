@@ -312,13 +312,12 @@ svdq_status launch_gemm_single(const svdq_shape& s, int rank, const void* Qx, co
   return SVDQ_OK;
 }
 
-constexpr int kPairStages = 5;
-
+template <int NB>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = svdq::PairSmem<kPairStages>::kBytes;
+  cfg.dynamicSmemBytes = svdq::PairCfg<NB>::kBytes;
   cfg.stream = st;
   attr->id = cudaLaunchAttributeClusterDimension;
   attr->val.clusterDim.x = 2;
@@ -329,20 +328,22 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
   return cfg;
 }
 
-// Clusters of the pair kernel that fit on the device at once (cached per device).
+// Clusters of the pair kernel (tile width NB) that fit on the device at once,
+// cached per device; also sets the kernel's shared-memory attribute there.
+template <int NB>
 int pair_clusters() {
   static int cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (dev < 64 && cached[dev]) return cached[dev];
-  auto kern = svdq::svdq_gemm_pair_kernel<kPairStages>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairSmem<kPairStages>::kBytes) !=
+  auto kern = svdq::svdq_gemm_pair_kernel<NB>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB>::kBytes) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config(sm_count() / 2, nullptr, &attr);
+  cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, &attr);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -352,25 +353,27 @@ int pair_clusters() {
   return n;
 }
 
+template <int NB>
 svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T,
                              const void* Qr, const void* Sr, const void* L2t, void* Y, cudaStream_t st,
                              int clusters) {
+  constexpr uint32_t kBBox = NB == 256 ? 128 : 64;   // B rows per TMA box
   CUtensorMap tqx, tqr, tsa, tsb, tt, tl, ty;
   svdq_status r;
   if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, svdq::kGemmBKBytes,
                      128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
     return r;
   if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.N, svdq::kGemmBKBytes,
-                     128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+                     kBBox, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
     return r;
   if ((r = make_scale_tmap(&tsa, Sx, s.M, s.K, 1)) != SVDQ_OK) return r;
-  if ((r = make_scale_tmap(&tsb, Sr, s.N, s.K, 2)) != SVDQ_OK) return r;
+  if ((r = make_scale_tmap(&tsb, Sr, s.N, s.K, NB / 128)) != SVDQ_OK) return r;
   if (rank > 0) {
     if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.M, svdq::kGemmLrK, 128,
                        CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
       return r;
     if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)rank, (uint64_t)s.N, svdq::kGemmLrK,
-                       128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+                       kBBox, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
       return r;
   } else {
     memset(&tt, 0, sizeof(tt));
@@ -379,25 +382,28 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
   if ((r = make_tmap(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)s.M, svdq::kEpiBoxCols, 32,
                      CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
     return r;
-  using L = svdq::PairSmem<kPairStages>;
-  auto kern = svdq::svdq_gemm_pair_kernel<kPairStages>;
-  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
-  const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / svdq::kPairBN);
+  auto kern = svdq::svdq_gemm_pair_kernel<NB>;
+  const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / NB);
   const int ncl = (int)(tiles < clusters ? tiles : clusters);
   cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config(ncl, st, &attr);
+  cudaLaunchConfig_t cfg = pair_config<NB>(ncl, st, &attr);
   SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank));
   SVDQ_LAUNCHED("svdq_gemm_pair_kernel");
   return SVDQ_OK;
 }
 
-// CTA-pair kernel when N is a multiple of 256 and pairs fit on the device,
-// otherwise the single-CTA kernel.
+// CTA pairs with 256 x 384 tiles when N is a multiple of 384, 256 x 256 tiles
+// when it is a multiple of 256, otherwise the single-CTA kernel (also when
+// pairs do not fit on the device).
 svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
                         const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
-  if (s.N % svdq::kPairBN == 0) {
-    const int clusters = pair_clusters();
-    if (clusters > 0) return launch_gemm_pair(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
+  if (s.N % 384 == 0) {
+    const int clusters = pair_clusters<384>();
+    if (clusters > 0) return launch_gemm_pair<384>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
+  }
+  if (s.N % 256 == 0) {
+    const int clusters = pair_clusters<256>();
+    if (clusters > 0) return launch_gemm_pair<256>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
   }
   return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
 }

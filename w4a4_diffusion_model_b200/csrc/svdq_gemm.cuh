@@ -240,13 +240,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
       tc_fence_after();
       if (!ok || device_error_set()) break;
       uint32_t p[64];
-      epilogue_drain_pack(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), p);
+      epilogue_drain_pack<4>(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), p);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);   // accumulator drained: the next tile may start
       const int col0 = n0 + h * 128;
       if (col0 >= N) continue;                 // second half of a 128-wide last column tile
-      epilogue_store_band(p, box, &tm_y, col0, m0 + 32 * q, lane, true);
+      epilogue_store_band<2>(p, box, &tm_y, col0, m0 + 32 * q, lane, true);
     }
     if (lane == 0) bulk_wait<0>();   // every store of this warp has completed
   }

@@ -50,9 +50,12 @@ constexpr int kEpiBoxBytes = 32 * kEpiBoxCols * 2;
 //      (the MMA reads column 4*kb + q at lane 32q+i: the scales of A row 32q+i)
 //   B: column 8*kb + c of lane 32q+i  <-  scales of B row 32c+i, i.e. word c of
 //      line i of B atom kb (c < 4) or of the second 128-row half (c >= 4)
-// which is the layout tcgen05.cp.32x128b.warpx4 would produce.
+// which is the layout tcgen05.cp.32x128b.warpx4 would produce. With a third
+// 128-row block of B (`sfb2`, for a second MMA of N = 128), its scales follow
+// at column 48 + 4*kb + c, laid out like A's.
 __device__ __forceinline__ void scales_to_tmem(uint32_t tmem, int q, int lane, const unsigned char* sfa,
-                                               const unsigned char* sfb0, const unsigned char* sfb1, uint32_t col) {
+                                               const unsigned char* sfb0, const unsigned char* sfb1, uint32_t col,
+                                               const unsigned char* sfb2 = nullptr) {
   uint32_t ra[16], rb[32];
 #pragma unroll
   for (int kb = 0; kb < kGemmKBPerStage; ++kb) {
@@ -66,13 +69,22 @@ __device__ __forceinline__ void scales_to_tmem(uint32_t tmem, int q, int lane, c
   const uint32_t t = tmem + ((uint32_t)(q * 32) << 16) + col;
   tmem_st_32x32b_x16(t, ra);
   tmem_st_32x32b_x32(t + 4 * kGemmKBPerStage, rb);
+  if (sfb2 != nullptr) {
+#pragma unroll
+    for (int kb = 0; kb < kGemmKBPerStage; ++kb) {
+      const uint4 b2 = *reinterpret_cast<const uint4*>(sfb2 + kb * kSfAtomBytes + lane * 16);
+      ra[4 * kb] = b2.x; ra[4 * kb + 1] = b2.y; ra[4 * kb + 2] = b2.z; ra[4 * kb + 3] = b2.w;
+    }
+    tmem_st_32x32b_x16(t + 12 * kGemmKBPerStage, ra);
+  }
 }
 
-// Drain 128 accumulator columns of this warp's lane band (32 at a time) and
-// pack them to bf16 pairs: p[j] holds columns 2j and 2j+1.
-__device__ __forceinline__ void epilogue_drain_pack(uint32_t taddr, uint32_t (&p)[64]) {
+// Drain 32 * CHUNKS accumulator columns of this warp's lane band (32 at a
+// time) and pack them to bf16 pairs: p[j] holds columns 2j and 2j+1.
+template <int CHUNKS>
+__device__ __forceinline__ void epilogue_drain_pack(uint32_t taddr, uint32_t (&p)[16 * CHUNKS]) {
 #pragma unroll
-  for (int c = 0; c < 4; ++c) {
+  for (int c = 0; c < CHUNKS; ++c) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(taddr + 32 * c, v);
     tmem_ld_wait();
@@ -84,13 +96,14 @@ __device__ __forceinline__ void epilogue_drain_pack(uint32_t taddr, uint32_t (&p
   }
 }
 
-// Write one warp's 32 x 128 bf16 band (row `lane` = p) as two 32 x 64 boxes
-// through a 128B-swizzled staging box and TMA stores (clipped at the edge).
-__device__ __forceinline__ void epilogue_store_band(const uint32_t (&p)[64], unsigned char* box, const void* tm_y,
-                                                    int col0, int row0, int lane, bool store) {
+// Write one warp's 32 x (64 * BOXES) bf16 band (row `lane` = p) as 32 x 64
+// boxes through a 128B-swizzled staging box and TMA stores (clipped at the edge).
+template <int BOXES>
+__device__ __forceinline__ void epilogue_store_band(const uint32_t (&p)[32 * BOXES], unsigned char* box,
+                                                    const void* tm_y, int col0, int row0, int lane, bool store) {
   const uint32_t box_addr = smem_u32(box);
 #pragma unroll
-  for (int b = 0; b < 2; ++b) {
+  for (int b = 0; b < BOXES; ++b) {
     if (lane == 0) bulk_wait_read<0>();   // the previous store from this box has read it
     __syncwarp();
 #pragma unroll

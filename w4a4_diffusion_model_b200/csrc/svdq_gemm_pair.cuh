@@ -1,17 +1,22 @@
 // The W4A4 GEMM on CTA pairs: one tcgen05 MMA (cta_group::2) spans the two
-// SMs of a cluster of 2, computing a 256 x 256 tile of
+// SMs of a cluster of 2, computing a 256 x NB tile (NB = 256 or 384) of
 //   Y = bf16( deq(Qx) deq(Qr)^T  +  T L2t^T )
 // (devpress.csdn.net SVDQuant walkthrough, eq. (2), eq. (5) and Fig. 6).
 // Each CTA of the pair stages its own 128 rows of the A operand (Qx, then T)
-// and its own 128 rows of the B operand (Qr, then L2t), so a pair reads 2/3 of
-// the operand bytes two independent 128 x 256 tiles would; each CTA also
-// stages the A scales of its rows and the B scales of all 256 columns, and its
-// scale warps write them into its own TMEM (the pair MMA reads both).
+// and its own NB/2 rows of the B operand (Qr, then L2t); each CTA also stages
+// the A scales of its rows and the B scales of all NB columns, and its scale
+// warps write them into its own TMEM (the pair MMA reads both).
+//
+// NB = 384 (two MMAs per K block: N = 256 into accumulator columns [0, 256),
+// N = 128 into [256, 384)) reads 16 % fewer operand bytes per FLOP than
+// NB = 256; its accumulator leaves room in TMEM for two scale buffers only,
+// used in turn (buffer it % 2 is free once the commit of item it - 2 landed).
+// With NB = 256 every ring stage has its own scale buffer.
 //
 // Persistent: cluster c walks pair tiles c, c + clusters, ... Each tile is a
 // sequence of items (K/256 FP4 k-tiles, then ceil(r/64) low-rank k-tiles).
 // Roles per CTA (448 threads), identical in both CTAs except where noted:
-//   warps 0-7   epilogue: drain this CTA's 128 x 256 fp32 accumulator,
+//   warps 0-7   epilogue: drain this CTA's 128 x NB fp32 accumulator,
 //               release it to the even CTA's MMA issuer, write Y through
 //               128B-swizzled boxes and TMA stores
 //   warp 8      producer: TMA loads of this CTA's item rows and scale atoms,
@@ -21,8 +26,8 @@
 //               reported it, and releases each ring stage (with its TMEM
 //               scale buffer) and the accumulator of both CTAs with
 //               multicast tcgen05.commit
-//   warps 10-13 scale warps: wait for this CTA's stage, put its scales in the
-//               stage's TMEM scale buffer (tcgen05.st), report to the even CTA
+//   warps 10-13 scale warps: wait for this CTA's stage, put its scales in a
+//               TMEM scale buffer (tcgen05.st), report to the even CTA
 // Every wait is bounded; on a timeout the kernel records a device error word,
 // every role stops, and both CTAs still meet at the final cluster barrier.
 #pragma once
@@ -35,34 +40,46 @@
 namespace svdq {
 
 constexpr int kPairBM = 256;                          // M rows per pair tile (128 per CTA)
-constexpr int kPairBN = 256;                          // N columns per pair tile (B rows: 128 per CTA)
 constexpr int kPairStageA = 128 * kGemmBKBytes;       // 16 KB: this CTA's 128 Qx rows (or T rows)
-constexpr int kPairStageB = 128 * kGemmBKBytes;       // 16 KB: this CTA's 128 Qr rows (or L2t rows)
 constexpr int kPairStageSfa = kGemmKBPerStage * kSfAtomBytes;       // 2 KB
-constexpr int kPairStageSfb = 2 * kGemmKBPerStage * kSfAtomBytes;   // 4 KB (both 128-row halves of N)
-constexpr int kPairStageBytes = kPairStageA + kPairStageB + kPairStageSfa + kPairStageSfb;   // 38 KB
 
-template <int STAGES>
-struct PairSmem {
-  static constexpr int kEpiOffset = STAGES * kPairStageBytes;
+template <int NB>
+struct PairCfg {
+  static_assert(NB == 256 || NB == 384, "pair tile width");
+  static constexpr int kBRows = NB / 2;                               // B rows per CTA
+  static constexpr int kStageB = kBRows * kGemmBKBytes;               // 16 | 24 KB
+  static constexpr int kSfbBlocks = NB / 128;                         // 128-row blocks of B scales
+  static constexpr int kStageSfb = kSfbBlocks * kGemmKBPerStage * kSfAtomBytes;   // 4 | 6 KB
+  static constexpr int kStageBytes = kPairStageA + kStageB + kPairStageSfa + kStageSfb;   // 38 | 48 KB
+  static constexpr int kStages = NB == 256 ? 5 : 4;
+  static constexpr uint32_t kSfCols = 4 * kGemmKBPerStage * (1 + kSfbBlocks);   // 48 | 64 TMEM columns
+  static constexpr int kSfBufs = (int)((kTmemCols - NB) / kSfCols);             // 5 | 2
+  static constexpr bool kSfPerStage = kSfBufs >= kStages;
+  static_assert(kSfBufs >= 2, "scale buffers");
+  static constexpr int kEpiOffset = kStages * kStageBytes;
   static constexpr int kBarOffset = kEpiOffset + kGemmEpiWarps * kEpiBoxBytes;
   static constexpr int kBytes = kBarOffset + 512 + 1024;
+  // TMEM column of the scale buffer of item `it` in ring stage `s`
+  __device__ static uint32_t sf_col(uint32_t it, int s) {
+    return (uint32_t)NB + (kSfPerStage ? (uint32_t)s : it % (uint32_t)kSfBufs) * kSfCols;
+  }
 };
 
 // Launched with a cluster dimension of (2, 1, 1).
+// tm_qr / tm_l2 boxes are 128 rows (NB = 256) or 64 rows (NB = 384).
 // tm_sfa / tm_sfb view a native scale buffer as 3-D uint8
-// [row blocks][K/64 * 2 chunks][256 bytes]; box {256, 8, 1|2} (4 atoms per row block).
-template <int STAGES>
+// [row blocks][K/64 * 2 chunks][256 bytes]; box {256, 8, 1 | NB/128} (4 atoms per row block).
+template <int NB>
 __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     const __grid_constant__ CUtensorMap tm_qx, const __grid_constant__ CUtensorMap tm_qr,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
     const __grid_constant__ CUtensorMap tm_y, int M, int N, int K, int rank) {
-  using L = PairSmem<STAGES>;
-  static_assert(STAGES <= kMaxSfBufs, "one TMEM scale buffer per ring stage");
+  using C = PairCfg<NB>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
   uint64_t* empty = full + STAGES;
   uint64_t* sf_ready = empty + STAGES;      // even CTA: both CTAs' scale warps report here
   uint64_t* acc_full = sf_ready + STAGES;
@@ -74,7 +91,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
   const uint32_t crank = cluster_ctarank();
   const bool leader = crank == 0;
   const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
-  const int tiles_n = N / kPairBN;
+  const int tiles_n = N / NB;
   const int ntiles = ((M + kPairBM - 1) / kPairBM) * tiles_n;
   const int kb_total = K >> 6;
   const int n_fp4_kt = (kb_total + kGemmKBPerStage - 1) / kGemmKBPerStage;
@@ -117,28 +134,40 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       bool ok = true;
       for (int tile = cluster; tile < ntiles && ok; tile += nclusters) {
         const int m0 = (tile / tiles_n) * kPairBM + 128 * (int)crank;   // this CTA's A rows
-        const int n0 = (tile % tiles_n) * kPairBN;                      // the pair's N columns
+        const int n0 = (tile % tiles_n) * NB;                           // the pair's N columns
         for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
           const int s = it % STAGES;
           if (!mbar_wait(empty + s, ((it / STAGES) & 1u) ^ 1u, kDevErrTimeoutEmpty)) {
             ok = false;
             break;
           }
-          unsigned char* sa = smem + s * kPairStageBytes;
+          unsigned char* sa = smem + s * C::kStageBytes;
           unsigned char* sb = sa + kPairStageA;
           if (kt < n_fp4_kt) {
-            unsigned char* sfa = sb + kPairStageB;
+            unsigned char* sfa = sb + C::kStageB;
             unsigned char* sfb = sfa + kPairStageSfa;
-            mbar_arrive_expect_tx(full + s, (uint32_t)kPairStageBytes);
+            mbar_arrive_expect_tx(full + s, (uint32_t)C::kStageBytes);
             tma_load_2d(sa, &tm_qx, full + s, kt * kGemmBKBytes, m0);
-            tma_load_2d(sb, &tm_qr, full + s, kt * kGemmBKBytes, n0 + 128 * (int)crank);
+            if (NB == 256) {
+              tma_load_2d(sb, &tm_qr, full + s, kt * kGemmBKBytes, n0 + 128 * (int)crank);
+            } else {   // rows n0 + 128 c + [0, 128) for the first MMA, n0 + 256 + 64 c + [0, 64) for the second
+              tma_load_2d(sb, &tm_qr, full + s, kt * kGemmBKBytes, n0 + 128 * (int)crank);
+              tma_load_2d(sb + 64 * kGemmBKBytes, &tm_qr, full + s, kt * kGemmBKBytes, n0 + 128 * (int)crank + 64);
+              tma_load_2d(sb + 128 * kGemmBKBytes, &tm_qr, full + s, kt * kGemmBKBytes, n0 + 256 + 64 * (int)crank);
+            }
             tma_load_3d(sfa, &tm_sfa, full + s, 0, kt * kGemmKBPerStage * 2, m0 >> 7);
             tma_load_3d(sfb, &tm_sfb, full + s, 0, kt * kGemmKBPerStage * 2, n0 >> 7);
           } else {
             const int c = kt - n_fp4_kt;
-            mbar_arrive_expect_tx(full + s, (uint32_t)(kPairStageA + kPairStageB));
+            mbar_arrive_expect_tx(full + s, (uint32_t)(kPairStageA + C::kStageB));
             tma_load_2d(sa, &tm_t, full + s, c * kGemmLrK, m0);
-            tma_load_2d(sb, &tm_l2, full + s, c * kGemmLrK, n0 + 128 * (int)crank);
+            if (NB == 256) {
+              tma_load_2d(sb, &tm_l2, full + s, c * kGemmLrK, n0 + 128 * (int)crank);
+            } else {
+              tma_load_2d(sb, &tm_l2, full + s, c * kGemmLrK, n0 + 128 * (int)crank);
+              tma_load_2d(sb + 64 * kGemmBKBytes, &tm_l2, full + s, c * kGemmLrK, n0 + 128 * (int)crank + 64);
+              tma_load_2d(sb + 128 * kGemmBKBytes, &tm_l2, full + s, c * kGemmLrK, n0 + 256 + 64 * (int)crank);
+            }
           }
         }
       }
@@ -156,17 +185,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     for (int tile = cluster; tile < ntiles && ok; tile += nclusters) {
       for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
         const int s = it % STAGES;
-        // stage s has landed; its scale buffer was freed by the commit that
-        // released the stage's previous use (which preceded this refill)
+        // stage s has landed
         if (!mbar_wait(full + s, (it / STAGES) & 1u, kDevErrTimeoutFull)) {
           ok = false;
           break;
         }
+        // its scale buffer is free: with one buffer per stage, the commit that
+        // released the stage's previous use (which preceded this refill) freed
+        // it; with buffers used in turn, wait for the commit of the buffer's
+        // previous item (items complete in order, so that phase of its stage's
+        // barrier is the latest one that can have completed)
+        if (!C::kSfPerStage && it >= (uint32_t)C::kSfBufs) {
+          const uint32_t pj = it - (uint32_t)C::kSfBufs;
+          if (!mbar_wait(empty + pj % STAGES, (pj / STAGES) & 1u, kDevErrTimeoutScales)) {
+            ok = false;
+            break;
+          }
+        }
         tc_fence_after();
         if (kt < n_fp4_kt) {
-          const unsigned char* sfa = smem + s * kPairStageBytes + kPairStageA + kPairStageB;
+          const unsigned char* sfa = smem + s * C::kStageBytes + kPairStageA + C::kStageB;
           const unsigned char* sfb = sfa + kPairStageSfa;
-          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + kPairStageSfb / 2, sf_buf_col(s));
+          scales_to_tmem(tmem, q, lane, sfa, sfb, sfb + 4 * kSfAtomBytes, C::sf_col(it, s),
+                         NB == 384 ? sfb + 8 * kSfAtomBytes : nullptr);
           tmem_st_wait();
         }
         tc_fence_before();
@@ -179,8 +220,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       // ---------------------------------------------------------------- MMA issuer (even CTA)
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      const uint32_t idesc = idesc_nvfp4(kPairBM, kPairBN);
-      const uint32_t idesc_lr = idesc_bf16(kPairBM, kPairBN);
+      const uint32_t idesc = idesc_nvfp4(kPairBM, 256);
+      const uint32_t idesc2 = idesc_nvfp4(kPairBM, 128);
+      const uint32_t idesc_lr = idesc_bf16(kPairBM, 256);
+      const uint32_t idesc_lr2 = idesc_bf16(kPairBM, 128);
       for (int tile = cluster; tile < ntiles && ok; tile += nclusters, ++tcount) {
         if (!mbar_wait_cluster(acc_empty, (tcount & 1u) ^ 1u, kDevErrTimeoutAccum)) {
           ok = false;
@@ -195,16 +238,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * kPairStageBytes);
+          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
           const uint32_t sb = sa + kPairStageA;
+          const uint32_t sb2 = sb + 128 * kGemmBKBytes;   // B rows of the second MMA (NB = 384)
           if (kt < n_fp4_kt) {
-            const uint32_t sfa = tmem + sf_buf_col(s);
+            const uint32_t sfa = tmem + C::sf_col(it, s);
             const uint32_t sfb = sfa + 4 * kGemmKBPerStage;
+            const uint32_t sfb2 = sfa + 12 * kGemmKBPerStage;
             const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
             for (int kb = 0; kb < kbs; ++kb) {
+              const uint32_t acc = (kt | kb) != 0 ? 1u : 0u;
               const uint64_t ad = smem_desc(sa + kb * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(sb + kb * 32, 16, 1024, kSwizzle128B);
-              mma_nvfp4_pair(tmem, ad, bd, idesc, sfa + 4 * kb, sfb + 8 * kb, (kt | kb) != 0 ? 1u : 0u);
+              mma_nvfp4_pair(tmem, ad, bd, idesc, sfa + 4 * kb, sfb + 8 * kb, acc);
+              if (NB == 384) {
+                const uint64_t bd2 = smem_desc(sb2 + kb * 32, 16, 1024, kSwizzle128B);
+                mma_nvfp4_pair(tmem + 256, ad, bd2, idesc2, sfa + 4 * kb, sfb2 + 4 * kb, acc);
+              }
             }
           } else {
             const int c = kt - n_fp4_kt;
@@ -213,6 +263,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
               const uint64_t ad = smem_desc(sa + j * 32, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(sb + j * 32, 16, 1024, kSwizzle128B);
               mma_bf16_pair(tmem, ad, bd, idesc_lr, 1u);
+              if (NB == 384) {
+                const uint64_t bd2 = smem_desc(sb2 + j * 32, 16, 1024, kSwizzle128B);
+                mma_bf16_pair(tmem + 256, ad, bd2, idesc_lr2, 1u);
+              }
             }
           }
           tc_commit_pair(empty + s, 0x3);     // stage s and its scale buffer, in both CTAs, are free
@@ -227,22 +281,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
   } else {
     // ------------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3, h = warp >> 2;
-    unsigned char* box = smem + L::kEpiOffset + warp * kEpiBoxBytes;
+    unsigned char* box = smem + C::kEpiOffset + warp * kEpiBoxBytes;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     if (lane == 0) prefetch_tmap(&tm_y);
     uint32_t tcount = 0;
     for (int tile = cluster; tile < ntiles; tile += nclusters, ++tcount) {
       const int m0 = (tile / tiles_n) * kPairBM + 128 * (int)crank;
-      const int n0 = (tile % tiles_n) * kPairBN;
+      const int n0 = (tile % tiles_n) * NB;
       const bool ok = mbar_wait(acc_full, tcount & 1u, kDevErrTimeoutAccum);
       tc_fence_after();
       if (!ok || device_error_set()) break;
+      // warp (q, h): lanes 32q.., accumulator columns h * NB/2 + [0, NB/2)
+      const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * (NB / 2));
+      const bool store = m0 + 32 * q < M;
       uint32_t p[64];
-      epilogue_drain_pack(tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128), p);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // this warp's part of the accumulator is drained
-      epilogue_store_band(p, box, &tm_y, n0 + h * 128, m0 + 32 * q, lane, m0 + 32 * q < M);
+      epilogue_drain_pack<4>(taddr, p);
+      if (NB == 256) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // this warp's part of the accumulator is drained
+        epilogue_store_band<2>(p, box, &tm_y, n0 + h * 128, m0 + 32 * q, lane, store);
+      } else {   // drain all 192 columns before releasing the accumulator, then store
+        uint32_t p2[32];
+        epilogue_drain_pack<2>(taddr + 128, p2);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        epilogue_store_band<2>(p, box, &tm_y, n0 + h * 192, m0 + 32 * q, lane, store);
+        epilogue_store_band<1>(p2, box, &tm_y, n0 + h * 192 + 128, m0 + 32 * q, lane, store);
+      }
     }
     if (lane == 0) bulk_wait<0>();
   }
