@@ -225,7 +225,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       const uint32_t idesc_lr = idesc_bf16(kPairBM, 256);
       const uint32_t idesc_lr2 = idesc_bf16(kPairBM, 128);
       for (int tile = cluster; tile < ntiles && ok; tile += nclusters, ++tcount) {
-        if (!mbar_wait_cluster(acc_empty, (tcount & 1u) ^ 1u, kDevErrTimeoutAccum)) {
+        // CTA-scope waits: the remote arrivals on acc_empty and sf_ready are
+        // relaxed and announce work already completed by its own mechanism
+        // (tcgen05.wait::ld / tcgen05.wait::st), so a cluster-scope acquire
+        // would order nothing and only costs issue time
+        if (!mbar_wait(acc_empty, (tcount & 1u) ^ 1u, kDevErrTimeoutAccum)) {
           ok = false;
           break;
         }
@@ -233,7 +237,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
           const int s = it % STAGES;
           // both CTAs' scale warps saw stage s full and put its scales in TMEM
-          if (!mbar_wait_cluster(sf_ready + s, (it / STAGES) & 1u, kDevErrTimeoutScales)) {
+          if (!mbar_wait(sf_ready + s, (it / STAGES) & 1u, kDevErrTimeoutScales)) {
             ok = false;
             break;
           }
