@@ -185,6 +185,29 @@ SVDQ_API svdq_status svdq_quantize_act(svdq_shape shape, const void* X, const fl
 SVDQ_API svdq_status svdq_linear(svdq_shape shape, const void* Qx, const void* Sx, const void* T, const void* Qr,
                         const void* Sr, const void* L2t, void* Y, int variant, void* stream);
 
+/* LoRA as part of the low-rank branch (walkthrough, Figure 9 and Figure 16: a
+ * LoRA runs in, or is merged into, the independent 16-bit branch, with no
+ * re-quantization of the residual). A LoRA update Y += X A^T B^T acts on the raw
+ * activation, exactly like the stored down-projection L1p (which already has
+ * lambda folded in), so the branch of rank r + extra is the concatenation
+ *   L1p_out [r + extra][K] = [L1p ; A],   L2t_out [N][r + extra] = [L2t , B].
+ * shape.K, shape.N, shape.rank = r describe the prepared layer (shape.M unused);
+ * L1p bf16 [r][K], L2t bf16 [N][r] (may be NULL when r == 0), A bf16 [extra][K],
+ * B bf16 [N][extra]. extra > 0, multiple of 16, r + extra <= 128
+ * (SVDQ_ERR_UNSUPPORTED_SHAPE otherwise). Outputs must not overlap the inputs.
+ * Qr/Sr are unchanged; use the layer with rank r + extra afterwards.
+ * Stream-ordered device copies only. */
+SVDQ_API svdq_status svdq_append_lowrank(svdq_shape shape, int32_t extra, const void* L1p, const void* L2t,
+                                         const void* A, const void* B, void* L1p_out, void* L2t_out,
+                                         void* stream);
+
+/* Diagnostic of the failure path (the pages have no counterpart): one thread
+ * waits, with the library's bounded wait, on a barrier phase that nothing
+ * completes; after the wait limit (2 s) it records the device error word and
+ * returns -- no fault, no hang, the context stays usable. The next svdq_check()
+ * on the stream returns SVDQ_ERR_TIMEOUT and clears the word. */
+SVDQ_API svdq_status svdq_selftest_timeout(void* stream);
+
 /* Native scale layout -> canonical [rows][K/16] bytes (inspection helper). */
 SVDQ_API svdq_status svdq_scales_to_canonical(int64_t rows, int64_t K, const void* native, void* canonical,
                                      void* stream);

@@ -97,6 +97,19 @@ def test_null_misaligned_and_variant_rejected(lib):
     assert b"aligned" in lib.svdq_last_error()
 
 
+def test_append_lowrank_argument_checks(lib):
+    good = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    sh = S.Shape(0, 256, 128, 32)
+    assert lib.svdq_append_lowrank(sh, 8, good, good, good, good, good, good, None) == 2      # not a multiple of 16
+    assert lib.svdq_append_lowrank(sh, 112, good, good, good, good, good, good, None) == 2    # 32 + 112 > 128
+    assert lib.svdq_append_lowrank(sh, 0, good, good, good, good, good, good, None) == 2
+    assert lib.svdq_append_lowrank(sh, 16, None, good, good, good, good, good, None) == 1     # L1p missing (r > 0)
+    assert lib.svdq_append_lowrank(sh, 16, good, good, bad, good, good, good, None) == 3
+    if not torch.cuda.is_available():   # r == 0: factors may be NULL; only the device check remains
+        assert lib.svdq_append_lowrank(S.Shape(0, 256, 128, 0), 16, None, None, good, good, good, good, None) == 5
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_no_device_is_reported_not_emulated(lib):
     sh = S.Shape(128, 256, 128, 0)

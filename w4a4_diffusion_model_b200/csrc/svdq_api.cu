@@ -707,6 +707,68 @@ svdq_status svdq_linear(svdq_shape s, const void* Qx, const void* Sx, const void
   return launch_up_rmw(s, s.rank, T, L2t, Y, st);
 }
 
+namespace svdq {
+
+// L2t_out[n][:r] = L2t[n], L2t_out[n][r:] = B[n]; 16-byte chunks (r, extra multiples of 16).
+__global__ void append_l2t_kernel(const uint4* __restrict__ L2t, const uint4* __restrict__ B, uint4* __restrict__ out,
+                                  int N, int r, int extra) {
+  const int cr = r / 8, ce = extra / 8, co = cr + ce;   // 8 bf16 per chunk
+  const size_t n_chunks = (size_t)N * co;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n_chunks; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t n = i / co;
+    const int c = (int)(i % co);
+    out[i] = c < cr ? L2t[n * cr + c] : B[n * ce + (c - cr)];
+  }
+}
+
+// One thread waits on a barrier phase that never completes; the bounded wait
+// gives up, records kDevErrSelfTest and the kernel returns.
+__global__ void selftest_timeout_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait(&bar, 0u, kDevErrSelfTest);   // gives up after kWaitLimitNs and records the code
+  }
+}
+
+}  // namespace svdq
+
+svdq_status svdq_append_lowrank(svdq_shape s, int32_t extra, const void* L1p, const void* L2t, const void* A,
+                                const void* B, void* L1p_out, void* L2t_out, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (extra <= 0 || extra % 16 || s.rank + extra > 128)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "rank %d + extra %d: need extra > 0, a multiple of 16, total <= 128",
+                (int)s.rank, (int)extra);
+  if (!A || !B || !L1p_out || !L2t_out || (s.rank > 0 && (!L1p || !L2t)))
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {L1p, L2t, A, B, L1p_out, L2t_out};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t l1_bytes = (size_t)s.rank * (size_t)s.K * 2u, a_bytes = (size_t)extra * (size_t)s.K * 2u;
+  if (l1_bytes) SVDQ_CUDA(cudaMemcpyAsync(L1p_out, L1p, l1_bytes, cudaMemcpyDeviceToDevice, st));
+  SVDQ_CUDA(cudaMemcpyAsync(static_cast<char*>(L1p_out) + l1_bytes, A, a_bytes, cudaMemcpyDeviceToDevice, st));
+  const size_t chunks = (size_t)s.N * (size_t)((s.rank + extra) / 8);
+  const unsigned grid = (unsigned)((chunks + 255) / 256 < 4096 ? (chunks + 255) / 256 : 4096);
+  svdq::append_l2t_kernel<<<grid, 256, 0, st>>>(static_cast<const uint4*>(L2t), static_cast<const uint4*>(B),
+                                                static_cast<uint4*>(L2t_out), (int)s.N, (int)s.rank, (int)extra);
+  SVDQ_LAUNCHED("append_l2t_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_selftest_timeout(void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_device();
+  if (r != SVDQ_OK) return r;
+  svdq::selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>();
+  SVDQ_LAUNCHED("selftest_timeout_kernel");
+  return SVDQ_OK;
+}
+
 svdq_status svdq_scales_to_canonical(int64_t rows, int64_t K, const void* native, void* canonical, void* stream) {
   g_last_error[0] = 0;
   if (rows < 0 || K < 64 || K % 64 || K > (1ll << 20) || rows > (1ll << 31) - 1)

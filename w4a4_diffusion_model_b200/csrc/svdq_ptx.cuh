@@ -20,6 +20,7 @@ enum DeviceError : unsigned int {
   kDevErrTimeoutAccum = 3,    // epilogue waited too long for the accumulator
   kDevErrTimeoutTmem = 4,     // waited too long for a TMEM allocation/free slot
   kDevErrTimeoutScales = 5,   // waited too long for a TMEM scale buffer (ready or free)
+  kDevErrSelfTest = 6,        // the diagnostic wait of svdq_selftest_timeout gave up (as it must)
 };
 
 // Bound on any spin-wait inside a kernel, in nanoseconds of %globaltimer.

@@ -30,7 +30,7 @@ STATUS = {
 EXPORTS = [
     "svdq_status_string", "svdq_last_error", "svdq_version", "svdq_act_sizes", "svdq_weight_sizes",
     "svdq_channel_amax", "svdq_prepare_weights", "svdq_prepare_weights_static", "svdq_quantize_act",
-    "svdq_linear", "svdq_scales_to_canonical", "svdq_check",
+    "svdq_linear", "svdq_append_lowrank", "svdq_selftest_timeout", "svdq_scales_to_canonical", "svdq_check",
 ]
 
 
@@ -70,6 +70,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_prepare_weights_static.argtypes = [Shape, vp, vp, ctypes.c_float, ctypes.c_uint, vp, vp, vp, vp, vp,
                                                 vp, vp]
     lib.svdq_prepare_weights_static.restype = st
+    lib.svdq_append_lowrank.argtypes = [Shape, ctypes.c_int32, vp, vp, vp, vp, vp, vp, vp]
+    lib.svdq_append_lowrank.restype = st
+    lib.svdq_selftest_timeout.argtypes = [vp]
+    lib.svdq_selftest_timeout.restype = st
     lib.svdq_quantize_act.argtypes = [Shape, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
     lib.svdq_quantize_act.restype = st
     lib.svdq_linear.argtypes = [Shape, vp, vp, vp, vp, vp, vp, vp, ctypes.c_int, vp]
@@ -197,6 +201,23 @@ def svdq_scales_to_canonical(native: torch.Tensor, rows: int, K: int) -> torch.T
     out = torch.empty(rows, K // 16, dtype=torch.uint8, device=native.device)
     _check(load().svdq_scales_to_canonical(rows, K, _ptr(native), _ptr(out), _stream()))
     return out
+
+
+def svdq_append_lowrank(W: PreparedWeights, A: torch.Tensor, B: torch.Tensor) -> PreparedWeights:
+    """Prepared weights whose low-rank branch also carries the LoRA update
+    X A^T B^T: A bf16 [extra][K], B bf16 [N][extra]. Qr/Sr are shared."""
+    K, N, r = W.shape.K, W.shape.N, W.shape.rank
+    extra = A.shape[0]
+    L1p = torch.empty(r + extra, K, dtype=torch.bfloat16, device=A.device)
+    L2t = torch.empty(N, r + extra, dtype=torch.bfloat16, device=A.device)
+    _check(load().svdq_append_lowrank(W.shape.c(), extra, _ptr(W.L1p), _ptr(W.L2t), _ptr(A), _ptr(B), _ptr(L1p),
+                                      _ptr(L2t), _stream()))
+    return PreparedWeights(LayerShape(0, K, N, r + extra), W.Qr, W.Sr, L1p, L2t, W.lam, W.inv_lam)
+
+
+def svdq_selftest_timeout() -> None:
+    """Launch the failure-path diagnostic (a bounded wait that gives up after 2 s)."""
+    _check(load().svdq_selftest_timeout(_stream()))
 
 
 def svdq_check() -> None:
