@@ -22,7 +22,9 @@
 // lane (r mod 16) + 32 (r div 16).
 //
 // With K split over a cluster of `ksplit` CTAs the partial sums of T are added
-// in cluster rank order through distributed shared memory.
+// in cluster rank order through distributed shared memory: each CTA pushes its
+// partial rows into the owning CTA's slots (or, for large ranks, peers read
+// them remotely from the drained ring).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -55,12 +57,19 @@ struct QuantSmem {
   static constexpr int kInv = kCols * 4;
   // 1 KB aligned stages: the 128B swizzle pattern repeats every 1024 bytes
   static constexpr int kStage = (kQStageXBytes + kL1 + kInv + 1023) / 1024 * 1024;
-  static constexpr int kStages = kQSmemBudget / kStage < kQMaxStages ? kQSmemBudget / kStage : kQMaxStages;
-  static constexpr int kBarOffset = kStages * kStage;
   static constexpr int kRedStride = RANK + 4;                  // fp32 partial T rows, padded against bank conflicts
-  static constexpr int kRed = BM * kRedStride * 4;             // reuses the ring
+  static constexpr int kRed = BM * kRedStride * 4;             // partial T of the K slices ([slice][row][col])
+  // The partial sums get a region of their own (peers push into it while this
+  // CTA may still be quantizing) when at least three stages still fit beside
+  // it; otherwise they reuse the drained ring.
+  static constexpr int kStagesSep = RANK > 0 ? (kQSmemBudget - kRed) / kStage : 0;
+  static constexpr bool kRedSeparate = kStagesSep >= 3;
+  static constexpr int kStagesMax = kRedSeparate ? kStagesSep : kQSmemBudget / kStage;
+  static constexpr int kStages = kStagesMax < kQMaxStages ? kStagesMax : kQMaxStages;
+  static constexpr int kRedOffset = kRedSeparate ? kStages * kStage : 0;
+  static constexpr int kBarOffset = kStages * kStage + (kRedSeparate ? (kRed + 1023) / 1024 * 1024 : 0);
   static constexpr uint32_t kTmemCols = RANK <= 32 ? 32 : RANK <= 64 ? 64 : 128;
-  static_assert(kRed <= kBarOffset, "partial sums must fit in the ring");
+  static_assert(kRedSeparate || kRed <= kStages * kStage, "partial sums must fit in the ring");
   static_assert(kStages >= 2, "ring too shallow");
   static constexpr int kBytes = kBarOffset + 256 + 1024;
 };
@@ -253,66 +262,133 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
 
   if constexpr (RANK > 0) {
     // ------------------------------------------------------------------ T from TMEM
-    __syncthreads();   // every role has left its loop: the ring is free once the MMAs are done
-    float* red = reinterpret_cast<float*>(smem);   // [BM rows][kRedStride], partial T of this K slice
-    if (warp < 4) {
-      // warp q reads TMEM lanes 32q..32q+31: rows 32q + lane (BM = 128) or 16q + lane, lane < 16 (BM = 64)
-      const bool live = BM == 128 || lane < 16;
-      const int r = BM == 128 ? 32 * warp + lane : 16 * warp + lane;
-      const bool acc_ok = mbar_wait(acc_bar, 0u, kDevErrTimeoutAccum);
-      tc_fence_after();
+    // warp q < 4 reads TMEM lanes 32q..32q+31: rows 32q + lane (BM = 128) or
+    // 16q + lane, lane < 16 (BM = 64) of this CTA's partial T
+    const bool live = BM == 128 || lane < 16;
+    const int r = BM == 128 ? 32 * warp + lane : 16 * warp + lane;
+    const int rows_per = BM / ksplit;                // rows whose T this CTA finalises
+    float* red = reinterpret_cast<float*>(smem + L::kRedOffset);
+    if constexpr (L::kRedSeparate) {
+      // Push: each CTA writes its partial rows straight into slot [kslice] of
+      // the owning CTA's region (owner of row r: r / rows_per), so one cluster
+      // barrier publishes everything and nothing is read remotely afterwards.
+      if (warp < 4) {
+        const bool acc_ok = mbar_wait(acc_bar, 0u, kDevErrTimeoutAccum);
+        tc_fence_after();
+        const int owner = r / rows_per, rr = r % rows_per;
+        const uint32_t dst = mapa_shared(smem_u32(red + (kslice * rows_per + rr) * L::kRedStride), (uint32_t)owner);
 #pragma unroll
-      for (int c = 0; c < RANK / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * warp) << 16) + 16u * c, v);
-        tmem_ld_wait();
-        if (!live || !acc_ok) continue;
-        if (ksplit == 1) {
-          if (m0 + r < M) {
-            uint32_t p[8];
+        for (int c = 0; c < RANK / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * warp) << 16) + 16u * c, v);
+          tmem_ld_wait();
+          if (!live || !acc_ok) continue;
+          if (ksplit == 1) {
+            if (m0 + r < M) {
+              uint32_t p[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const __nv_bfloat162 bb = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-              p[i] = *reinterpret_cast<const uint32_t*>(&bb);
+              for (int i = 0; i < 8; ++i) {
+                const __nv_bfloat162 bb =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                p[i] = *reinterpret_cast<const uint32_t*>(&bb);
+              }
+              uint4* out = reinterpret_cast<uint4*>(T + (size_t)(m0 + r) * RANK + 16 * c);
+              out[0] = make_uint4(p[0], p[1], p[2], p[3]);
+              out[1] = make_uint4(p[4], p[5], p[6], p[7]);
             }
-            uint4* dst = reinterpret_cast<uint4*>(T + (size_t)(m0 + r) * RANK + 16 * c);
-            dst[0] = make_uint4(p[0], p[1], p[2], p[3]);
-            dst[1] = make_uint4(p[4], p[5], p[6], p[7]);
-          }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(red + r * L::kRedStride + 16 * c);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+            for (int i = 0; i < 4; ++i)
+              asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + 64u * c + 16u * i),
+                           "f"(__uint_as_float(v[4 * i])), "f"(__uint_as_float(v[4 * i + 1])),
+                           "f"(__uint_as_float(v[4 * i + 2])), "f"(__uint_as_float(v[4 * i + 3]))
+                           : "memory");
+          }
         }
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (warp == L::kMmaWarp) {
-      tc_fence_after();
-      tmem_dealloc(tmem, L::kTmemCols);
-    }
-    if (ksplit > 1) {
-      cluster_sync();
-      // CTA kslice finalises rows [kslice * BM / ksplit, ...), adding the slices in rank order
-      const int rows_per = BM / ksplit;
-      const int e0 = kslice * rows_per * RANK, e1 = e0 + rows_per * RANK;
-      const uint32_t red_addr = smem_u32(red);
-      for (int e = e0 + (int)threadIdx.x; e < e1; e += L::kThreads) {
-        const int row = e / RANK, col = e % RANK;
-        const uint32_t off = 4u * (uint32_t)(row * L::kRedStride + col);
-        float sum = 0.f;
-        for (int p = 0; p < ksplit; ++p) {
-          float x;
-          const uint32_t a = mapa_shared(red_addr + off, (uint32_t)p);
-          asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(a) : "memory");
-          sum += x;
-        }
-        if (m0 + row < M) T[(size_t)(m0 + row) * RANK + col] = __float2bfloat16_rn(sum);
+      tc_fence_before();
+      if (ksplit > 1) cluster_sync(); else __syncthreads();   // pushes visible; TMEM reads done
+      if (warp == L::kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
       }
-      cluster_sync();   // peers keep their partial sums until everyone has read them
+      if (ksplit > 1) {   // add the slices in rank order, from this CTA's own region
+        const int cols4 = RANK / 4;
+        for (int e = threadIdx.x; e < rows_per * cols4; e += L::kThreads) {
+          const int row = e / cols4, c4 = (e % cols4) * 4;
+          float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int p = 0; p < ksplit; ++p) {
+            const float4 x = *reinterpret_cast<const float4*>(red + (p * rows_per + row) * L::kRedStride + c4);
+            sum.x += x.x; sum.y += x.y; sum.z += x.z; sum.w += x.w;
+          }
+          const int grow = m0 + kslice * rows_per + row;
+          if (grow < M) {
+            const __nv_bfloat162 lo = __floats2bfloat162_rn(sum.x, sum.y), hi = __floats2bfloat162_rn(sum.z, sum.w);
+            *reinterpret_cast<uint2*>(T + (size_t)grow * RANK + c4) =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+          }
+        }
+      }
+    } else {
+      // Pull (large ranks): the partial rows reuse the drained ring; peers read
+      // them remotely after a cluster barrier and keep them until a second one.
+      __syncthreads();   // every role has left its loop: the ring is free once the MMAs are done
+      if (warp < 4) {
+        const bool acc_ok = mbar_wait(acc_bar, 0u, kDevErrTimeoutAccum);
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < RANK / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + ((uint32_t)(32 * warp) << 16) + 16u * c, v);
+          tmem_ld_wait();
+          if (!live || !acc_ok) continue;
+          if (ksplit == 1) {
+            if (m0 + r < M) {
+              uint32_t p[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const __nv_bfloat162 bb =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                p[i] = *reinterpret_cast<const uint32_t*>(&bb);
+              }
+              uint4* out = reinterpret_cast<uint4*>(T + (size_t)(m0 + r) * RANK + 16 * c);
+              out[0] = make_uint4(p[0], p[1], p[2], p[3]);
+              out[1] = make_uint4(p[4], p[5], p[6], p[7]);
+            }
+          } else {
+            float4* dst = reinterpret_cast<float4*>(red + r * L::kRedStride + 16 * c);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                   __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncthreads();
+      if (warp == L::kMmaWarp) {
+        tc_fence_after();
+        tmem_dealloc(tmem, L::kTmemCols);
+      }
+      if (ksplit > 1) {
+        cluster_sync();
+        // CTA kslice finalises rows [kslice * BM / ksplit, ...), adding the slices in rank order
+        const int e0 = kslice * rows_per * RANK, e1 = e0 + rows_per * RANK;
+        const uint32_t red_addr = smem_u32(red);
+        for (int e = e0 + (int)threadIdx.x; e < e1; e += L::kThreads) {
+          const int row = e / RANK, col = e % RANK;
+          const uint32_t off = 4u * (uint32_t)(row * L::kRedStride + col);
+          float sum = 0.f;
+          for (int p = 0; p < ksplit; ++p) {
+            float x;
+            const uint32_t a = mapa_shared(red_addr + off, (uint32_t)p);
+            asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(x) : "r"(a) : "memory");
+            sum += x;
+          }
+          if (m0 + row < M) T[(size_t)(m0 + row) * RANK + col] = __float2bfloat16_rn(sum);
+        }
+        cluster_sync();   // peers keep their partial sums until everyone has read them
+      }
     }
   }
 }
