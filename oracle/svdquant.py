@@ -54,6 +54,8 @@ __all__ = [
     "quantize_act", "linear", "layer_reference",
     "fake_quant_int", "smooth_fp", "svdquant_fakequant",
     "quant_error", "prop41_bound", "rel_fro", "fro",
+    "INT4_QMAX", "INT4_GROUP", "fp16", "quantize_int4", "dequantize_int4", "pack_int4", "unpack_int4",
+    "layer_reference_int4",
 ]
 
 # ---------------------------------------------------------------------------
@@ -339,6 +341,84 @@ def layer_reference(X, W_lin, alpha: float, rank: int, act_amax=None) -> dict:
 # and SVDQuant sections), used to pin the smoothing orientation and the SVD
 # split against the printed error tables.
 # ---------------------------------------------------------------------------
+
+# ---------------------------------------------------------------------------
+# INT4 W4A4 variant (the pages' path for GPUs without NVFP4: [P2] eq. (1) with
+# q_max = 2^(k-1) - 1 = 7 for signed 4-bit integers; [P3] "one scale per 64
+# elements"). Readings: fp16 scales, s = fp16_RNE(fp32(amax / 7)) saturating at
+# 65504; q = clamp(RNE(fp32(v * fp32(1/s))), -7, 7) (the same multiply-by-the-
+# rounded-reciprocal recipe as the NVFP4 codes); a zero scale gives zero codes.
+
+INT4_QMAX = 7
+INT4_GROUP = 64
+
+
+def fp16(v) -> np.ndarray:
+    """IEEE binary16 round-to-nearest-even (10-bit fraction, emin -14), saturating at 65504."""
+    return round_to_format(v, 10, -14, 65504.0)
+
+
+def quantize_int4(v32: np.ndarray, group: int = INT4_GROUP) -> tuple[np.ndarray, np.ndarray]:
+    """Symmetric INT4 group quantization along the last axis of fp32 values.
+
+    Returns (codes int8 in [-7, 7], scales as fp16 values in float64 [.., K/group])."""
+    v = np.asarray(v32, dtype=np.float64)
+    rows, K = v.shape
+    assert K % group == 0
+    g = v.reshape(rows, K // group, group)
+    amax = np.max(np.abs(g), axis=2)
+    s = fp16(fp32(amax / INT4_QMAX))
+    s = np.where(np.isinf(s), 65504.0, s)                    # saturate the scale
+    with np.errstate(divide="ignore"):
+        inv = fp32(np.where(s > 0, 1.0 / np.where(s > 0, s, 1.0), 0.0))
+    y = fp32(g * inv[:, :, None])
+    q = np.clip(np.rint(y), -INT4_QMAX, INT4_QMAX)            # np.rint rounds half to even
+    q = np.where(s[:, :, None] > 0, q, 0.0)
+    return q.reshape(rows, K).astype(np.int8), s
+
+
+def dequantize_int4(codes: np.ndarray, scales: np.ndarray, group: int = INT4_GROUP) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.float64)
+    rows, K = c.shape
+    return (c.reshape(rows, K // group, group) * np.asarray(scales, np.float64)[:, :, None]).reshape(rows, K)
+
+
+def pack_int4(codes: np.ndarray) -> np.ndarray:
+    """Two's-complement nibbles, element 2i in the low nibble of byte i."""
+    u = (np.asarray(codes, dtype=np.int16) & 0xF).astype(np.uint8)
+    return (u[:, 0::2] | (u[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_int4(packed: np.ndarray) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    lo = (p & 0xF).astype(np.int16)
+    hi = (p >> 4).astype(np.int16)
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty((p.shape[0], 2 * p.shape[1]), dtype=np.int8)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def layer_reference_int4(X, W_lin, alpha: float, rank: int, act_amax=None) -> dict:
+    """The same layer with INT4 (g = 64, fp16 scales) in place of NVFP4: the
+    smoothing and the stored low-rank factors are those of prepare_weights; the
+    residual R and the smoothed activation are INT4-quantized along K."""
+    X = np.asarray(X, dtype=np.float64)
+    if act_amax is None:
+        act_amax = channel_amax(X)
+    P = prepare_weights(W_lin, act_amax, alpha, rank)
+    Qr, Sr = quantize_int4(P["R32"].T)                        # [N][K], grouped along K
+    X32 = np.asarray(X, dtype=np.float32)
+    xhat = X32 * np.asarray(P["inv32"], dtype=np.float32)[None, :]
+    Qx, Sx = quantize_int4(xhat)
+    T = X @ P["L1p"] if rank else np.zeros((X.shape[0], 0))
+    Y = dequantize_int4(Qx, Sx) @ dequantize_int4(Qr, Sr).T
+    if rank:
+        Y = Y + T @ P["L2"]
+    return {**P, "Qx4": Qx, "Sx4": Sx, "Qr4": Qr, "Sr4": Sr, "T": T, "Y": Y, "Y_exact": X @ np.asarray(W_lin, np.float64).T}
+
 
 def fake_quant_int(x: np.ndarray, bits: int, axis=None) -> np.ndarray:
     """Symmetric uniform quantize-dequantize: s = max|x| / (2^(b-1) - 1) per
