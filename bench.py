@@ -250,6 +250,41 @@ def cpu_cores() -> int:
         return os.cpu_count() or 1
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def square_gemm_rate(S, dev, n=8192, reps=10) -> dict:
+    """The GEMM alone at rank 0 on a large square shape (n x n x n): the best
+    FP4 rate this kernel reaches -- an achieved figure, not a peak."""
+    g = torch.Generator(device="cpu").manual_seed(7)
+    X = (torch.randn(n, n, generator=g) / 4).to(torch.bfloat16).to(dev)
+    W = (torch.randn(n, n, generator=g) / n ** 0.5).to(torch.bfloat16).to(dev)
+    P = S.svdq_prepare_weights(W, S.svdq_channel_amax(X), 0.5, 0)
+    Qx, Sx, _ = S.svdq_quantize_act(X, P.inv_lam, None, 0, n)
+    Y = torch.empty(n, n, dtype=torch.bfloat16, device=dev)
+    for _ in range(3):
+        S.svdq_linear(Qx, Sx, None, P, out=Y)
+    best = float("inf")
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        S.svdq_linear(Qx, Sx, None, P, out=Y)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    S.svdq_check()
+    return {"shape": f"{n}x{n}x{n}", "ms": round(best, 4), "tflops": round(2 * n ** 3 / (best * 1e-3) / 1e12, 1),
+            "note": "achieved, not peak"}
+
+
 def time_cpu(fn, flops, seconds):
     fn()  # warm
     t0 = time.perf_counter()
@@ -462,9 +497,17 @@ def run_ours(args):
             ev[1].record(stream)
             ev[2].record(stream)
         kc, _ = timed(n_x, cublas)
+        # warm L2: the same inputs every step (no rotation)
+        k1w, k2w = timed(n_x, lambda i, ev: step(0, ev=ev))
         lay = statistics.mean(step_ms)
         lay_f = statistics.mean(a + b for a, b in zip(k1f, k2f))
+        q10, q50, q90 = np.percentile(step_ms, [10, 50, 90])
         extras = {
+            "layer_ms_p10_p50_p90": [round(float(q10), 4), round(float(q50), 4), round(float(q90), 4)],
+            "warm_l2_layer_ms": round(statistics.mean(a + b for a, b in zip(k1w, k2w)), 4),
+            "warm_l2_quantize_ms": round(statistics.mean(k1w), 4),
+            "warm_l2_gemm_ms": round(statistics.mean(k2w), 4),
+            "gemm_square_rank0": square_gemm_rate(S, dev),
             "prepare_ms_offline": round(prepare_ms, 3),
             "quantize_ms": round(k1_ms, 4), "gemm_ms": round(k2_ms, 4), "layer_ms": round(lay, 4),
             "unfused_layer_ms": round(statistics.mean(a + b for a, b in zip(k1u, k2u)), 4),
@@ -502,7 +545,14 @@ def run_ours(args):
             fn, fl, sample = oracle_sample(w, X_cpu, W_cpu)
             v, n, el = time_cpu(fn, fl, args.cpu_seconds)
             cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
-                   "sample": sample, "repeats": n, "seconds": round(el, 2)}
+                   "sample": sample, "repeats": n, "seconds": round(el, 2), "cpu_model": cpu_model()}
+            try:
+                from threadpoolctl import threadpool_limits
+                with threadpool_limits(limits=1):
+                    v1, _, _ = time_cpu(fn, fl, max(1.0, args.cpu_seconds / 4))
+                cpu["value_1_core"] = round(v1, 6)
+            except Exception as e:  # the single-core figure is informative only
+                cpu["value_1_core"] = f"unavailable: {type(e).__name__}"
 
     if rank_id == 0:
         line = {
