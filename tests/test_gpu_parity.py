@@ -34,7 +34,9 @@ def _inputs(M, K, N, rank, seed, outliers="first4"):
 
 
 CASES = [
-    # M, K, N, rank        N % 256 == 0 runs the CTA-pair GEMM, otherwise the single-CTA one
+    # M, K, N, rank        N % 256 == 0 runs the CTA-pair GEMM on 256 x 256 tiles, N % 384 == 0
+    # (not % 256) on 256 x 384 tiles, otherwise the single-CTA one; small M takes the single-CTA
+    # kernel when it keeps 1.5x as many SMs busy
     (256, 512, 512, 16),      # the tiny layer
     (200, 384, 256, 32),      # ragged M, K % 256 == 128
     (1, 128, 128, 0),         # one row, no branch
@@ -43,6 +45,7 @@ CASES = [
     (130, 256, 512, 128),     # maximum rank, ragged M, CTA pair
     (300, 384, 768, 32),      # ragged M and K on a CTA pair
     (512, 1024, 640, 48),
+    (3000, 256, 1920, 32),    # ragged M on 256 x 384 pair tiles (two MMAs per K block, scale buffers in turn)
 ]
 
 

@@ -392,28 +392,30 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
   return SVDQ_OK;
 }
 
-// CTA pairs with 256 x 384 tiles when N is a multiple of 384, 256 x 256 tiles
-// when it is a multiple of 256, otherwise the single-CTA kernel (also when
-// pairs do not fit on the device). For small M the pair tiles leave most SMs
+// CTA pairs with 256 x 256 tiles when N is a multiple of 256, 256 x 384 tiles
+// when it is a multiple of 384 only, otherwise the single-CTA kernel (also
+// when pairs do not fit on the device). The 256-wide tiles keep a TMEM scale
+// buffer per ring stage and measured as fast as or faster than the 384-wide
+// ones on the FLUX projections. For small M the pair tiles leave most SMs
 // idle; the single-CTA kernel's 128 x 256 tiles then occupy more of them, so
 // it is chosen when it keeps at least 1.5x as many SMs busy.
 svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
                         const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
   const long long sms = sm_count();
   const long long rows256 = (s.M + 255) / 256, rows128 = (s.M + 127) / 128;
-  const int nb = s.N % 384 == 0 ? 384 : s.N % 256 == 0 ? 256 : 0;
+  const int nb = s.N % 256 == 0 ? 256 : s.N % 384 == 0 ? 384 : 0;
   if (nb) {
     const long long pair_sms = 2 * rows256 * (s.N / nb), single_ctas = rows128 * ((s.N + 255) / 256);
     const long long busy_pair = pair_sms < sms ? pair_sms : sms, busy_single = single_ctas < sms ? single_ctas : sms;
     if (2 * busy_single >= 3 * busy_pair) return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
   }
+  if (nb == 256) {
+    const int clusters = pair_clusters<256>();
+    if (clusters > 0) return launch_gemm_pair<256>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
+  }
   if (s.N % 384 == 0) {
     const int clusters = pair_clusters<384>();
     if (clusters > 0) return launch_gemm_pair<384>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
-  }
-  if (s.N % 256 == 0) {
-    const int clusters = pair_clusters<256>();
-    if (clusters > 0) return launch_gemm_pair<256>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
   }
   return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
 }

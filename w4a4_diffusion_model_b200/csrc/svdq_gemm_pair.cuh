@@ -218,12 +218,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
   } else if (warp == kMmaWarp) {
     if (lane == 0 && leader) {
       // ---------------------------------------------------------------- MMA issuer (even CTA)
-      uint32_t it = 0, tcount = 0;
+      // The issuing thread runs only a few MMAs ahead of the tensor pipe, so
+      // every cycle it spends between two items' MMAs can leave the pipe idle.
+      // The loop is kept short: the stage index and barrier parity are carried
+      // from item to item, the shared-memory descriptors are offsets of two
+      // precomputed ones, and whether the next item's scales are in place is
+      // tested before this item's MMAs are queued, so that in the common case
+      // no barrier wait stands between two items.
+      uint32_t tcount = 0;
       bool ok = true;
       const uint32_t idesc = idesc_nvfp4(kPairBM, 256);
       const uint32_t idesc2 = idesc_nvfp4(kPairBM, 128);
       const uint32_t idesc_lr = idesc_bf16(kPairBM, 256);
       const uint32_t idesc_lr2 = idesc_bf16(kPairBM, 128);
+      // descriptors of stage 0; a stage, a 64-element K block (32 bytes) and
+      // the B rows of the second MMA are offsets of the 16-byte address field
+      // (shared addresses stay below 2^18, so the field cannot carry over)
+      const uint64_t dA0 = smem_desc(smem_u32(smem), 16, 1024, kSwizzle128B);
+      const uint64_t dB0 = smem_desc(smem_u32(smem) + kPairStageA, 16, 1024, kSwizzle128B);
+      constexpr uint32_t kStageDesc = (uint32_t)C::kStageBytes >> 4;
+      constexpr uint32_t kB2Desc = (128u * kGemmBKBytes) >> 4;
+      constexpr uint32_t kKbDesc = 32u >> 4;
+      const int n_items = n_fp4_kt + n_lr_kt;
+      int s = 0;                 // ring stage and barrier parity of the current item
+      uint32_t ph = 0;
+      uint32_t sfbuf = 0;        // item index mod 2 (scale buffers used in turn)
+      bool ready = false;        // the current item's stage and scales are known to be in place
       for (int tile = cluster; tile < ntiles && ok; tile += nclusters, ++tcount) {
         // CTA-scope waits: the remote arrivals on acc_empty and sf_ready are
         // relaxed and announce work already completed by its own mechanism
@@ -233,49 +253,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
           ok = false;
           break;
         }
-        tc_fence_after();
-        for (int kt = 0; kt < n_fp4_kt + n_lr_kt; ++kt, ++it) {
-          const int s = it % STAGES;
+        for (int kt = 0; kt < n_items; ++kt) {
           // both CTAs' scale warps saw stage s full and put its scales in TMEM
-          if (!mbar_wait(sf_ready + s, (it / STAGES) & 1u, kDevErrTimeoutScales)) {
+          if (!ready && !mbar_wait(sf_ready + s, ph, kDevErrTimeoutScales)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(smem + s * C::kStageBytes);
-          const uint32_t sb = sa + kPairStageA;
-          const uint32_t sb2 = sb + 128 * kGemmBKBytes;   // B rows of the second MMA (NB = 384)
+          const int s1 = s + 1 == STAGES ? 0 : s + 1;
+          const uint32_t ph1 = s + 1 == STAGES ? ph ^ 1u : ph;
+          ready = mbar_test(sf_ready + s1, ph1);
+          const uint64_t ad = dA0 + (uint64_t)((uint32_t)s * kStageDesc);
+          const uint64_t bd = dB0 + (uint64_t)((uint32_t)s * kStageDesc);
           if (kt < n_fp4_kt) {
-            const uint32_t sfa = tmem + C::sf_col(it, s);
+            const uint32_t sfa = tmem + (uint32_t)NB + (C::kSfPerStage ? (uint32_t)s : sfbuf) * C::kSfCols;
             const uint32_t sfb = sfa + 4 * kGemmKBPerStage;
             const uint32_t sfb2 = sfa + 12 * kGemmKBPerStage;
             const int kbs = min(kGemmKBPerStage, kb_total - kt * kGemmKBPerStage);
-            for (int kb = 0; kb < kbs; ++kb) {
-              const uint32_t acc = (kt | kb) != 0 ? 1u : 0u;
-              const uint64_t ad = smem_desc(sa + kb * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(sb + kb * 32, 16, 1024, kSwizzle128B);
-              mma_nvfp4_pair(tmem, ad, bd, idesc, sfa + 4 * kb, sfb + 8 * kb, acc);
-              if (NB == 384) {
-                const uint64_t bd2 = smem_desc(sb2 + kb * 32, 16, 1024, kSwizzle128B);
-                mma_nvfp4_pair(tmem + 256, ad, bd2, idesc2, sfa + 4 * kb, sfb2 + 4 * kb, acc);
+#pragma unroll
+            for (int kb = 0; kb < kGemmKBPerStage; ++kb) {
+              if (kb < kbs) {
+                const uint32_t acc = (kt | kb) != 0 ? 1u : 0u;
+                mma_nvfp4_pair(tmem, ad + kb * kKbDesc, bd + kb * kKbDesc, idesc, sfa + 4 * kb, sfb + 8 * kb, acc);
+                if (NB == 384)
+                  mma_nvfp4_pair(tmem + 256, ad + kb * kKbDesc, bd + kB2Desc + kb * kKbDesc, idesc2, sfa + 4 * kb,
+                                 sfb2 + 4 * kb, acc);
               }
             }
           } else {
-            const int c = kt - n_fp4_kt;
-            const int k16 = min(kGemmLrK, rank - c * kGemmLrK) / 16;
-            for (int j = 0; j < k16; ++j) {
-              const uint64_t ad = smem_desc(sa + j * 32, 16, 1024, kSwizzle128B);
-              const uint64_t bd = smem_desc(sb + j * 32, 16, 1024, kSwizzle128B);
-              mma_bf16_pair(tmem, ad, bd, idesc_lr, 1u);
-              if (NB == 384) {
-                const uint64_t bd2 = smem_desc(sb2 + j * 32, 16, 1024, kSwizzle128B);
-                mma_bf16_pair(tmem + 256, ad, bd2, idesc_lr2, 1u);
+            const int k16 = min(kGemmLrK, rank - (kt - n_fp4_kt) * kGemmLrK) / 16;
+#pragma unroll
+            for (int j = 0; j < kGemmLrK / 16; ++j) {
+              if (j < k16) {
+                mma_bf16_pair(tmem, ad + j * kKbDesc, bd + j * kKbDesc, idesc_lr, 1u);
+                if (NB == 384) mma_bf16_pair(tmem + 256, ad + j * kKbDesc, bd + kB2Desc + j * kKbDesc, idesc_lr2, 1u);
               }
             }
           }
           tc_commit_pair(empty + s, 0x3);     // stage s and its scale buffer, in both CTAs, are free
+          sfbuf ^= 1u;
+          s = s1;
+          ph = ph1;
         }
-        tc_commit_pair(acc_full, 0x3);        // both halves of the tile's accumulator are complete
+        if (ok) tc_commit_pair(acc_full, 0x3);   // both halves of the tile's accumulator are complete
       }
       if (!ok) {
         tc_commit_pair(mma_drain, 0x1);
