@@ -330,13 +330,13 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
 
 // Clusters of the pair kernel (tile width NB) that fit on the device at once,
 // cached per device; also sets the kernel's shared-memory attribute there.
-template <int NB>
+template <int NB, bool QNEXT = false>
 int pair_clusters() {
   static int cached[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
   if (dev < 64 && cached[dev]) return cached[dev];
-  auto kern = svdq::svdq_gemm_pair_kernel<NB>;
+  auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB>::kBytes) !=
       cudaSuccess) {
     cudaGetLastError();
@@ -353,10 +353,10 @@ int pair_clusters() {
   return n;
 }
 
-template <int NB>
+template <int NB, bool QNEXT = false>
 svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T,
                              const void* Qr, const void* Sr, const void* L2t, void* Y, cudaStream_t st,
-                             int clusters) {
+                             int clusters, const svdq::NextQuant& nq = svdq::NextQuant{}, bool store_y = true) {
   constexpr uint32_t kBBox = NB == 256 ? 128 : 64;   // B rows per TMA box
   CUtensorMap tqx, tqr, tsa, tsb, tt, tl, ty;
   svdq_status r;
@@ -379,15 +379,20 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
     memset(&tt, 0, sizeof(tt));
     memset(&tl, 0, sizeof(tl));
   }
-  if ((r = make_tmap(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)s.M, svdq::kEpiBoxCols, 32,
-                     CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
-    return r;
-  auto kern = svdq::svdq_gemm_pair_kernel<NB>;
+  if (store_y) {
+    if ((r = make_tmap(&ty, Y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)s.M, svdq::kEpiBoxCols,
+                       32, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+  } else {
+    memset(&ty, 0, sizeof(ty));
+  }
+  auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
   const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / NB);
   const int ncl = (int)(tiles < clusters ? tiles : clusters);
   cudaLaunchAttribute attr;
   cudaLaunchConfig_t cfg = pair_config<NB>(ncl, st, &attr);
-  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank));
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank, nq,
+                               store_y ? 1 : 0));
   SVDQ_LAUNCHED("svdq_gemm_pair_kernel");
   return SVDQ_OK;
 }
@@ -399,25 +404,42 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
 // ones on the FLUX projections. For small M the pair tiles leave most SMs
 // idle; the single-CTA kernel's 128 x 256 tiles then occupy more of them, so
 // it is chosen when it keeps at least 1.5x as many SMs busy.
-svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
-                        const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+// Which GEMM kernel serves shape s on the current device: 256 or 384 (CTA
+// pairs with that tile width) or 128 (the single-CTA kernel).
+int gemm_choice(const svdq_shape& s) {
   const long long sms = sm_count();
   const long long rows256 = (s.M + 255) / 256, rows128 = (s.M + 127) / 128;
   const int nb = s.N % 256 == 0 ? 256 : s.N % 384 == 0 ? 384 : 0;
   if (nb) {
     const long long pair_sms = 2 * rows256 * (s.N / nb), single_ctas = rows128 * ((s.N + 255) / 256);
     const long long busy_pair = pair_sms < sms ? pair_sms : sms, busy_single = single_ctas < sms ? single_ctas : sms;
-    if (2 * busy_single >= 3 * busy_pair) return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
+    if (2 * busy_single >= 3 * busy_pair) return 128;
   }
-  if (nb == 256) {
-    const int clusters = pair_clusters<256>();
-    if (clusters > 0) return launch_gemm_pair<256>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
+  if (nb == 256 && pair_clusters<256>() > 0) return 256;
+  if (s.N % 384 == 0 && pair_clusters<384>() > 0) return 384;
+  return 128;
+}
+
+svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                        const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+  switch (gemm_choice(s)) {
+    case 256: return launch_gemm_pair<256>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<256>());
+    case 384: return launch_gemm_pair<384>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<384>());
+    default: return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
   }
-  if (s.N % 384 == 0) {
-    const int clusters = pair_clusters<384>();
-    if (clusters > 0) return launch_gemm_pair<384>(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, clusters);
-  }
-  return launch_gemm_single(s, rank, Qx, Sx, T, Qr, Sr, L2t, Y, st);
+}
+
+// The next layer's quantization runs in the GEMM epilogue when the next layer
+// has no low-rank branch and the shape takes the 256 x 256 pair kernel; every
+// other case forms Y (in the caller's Y or in the workspace) and runs the
+// quantizer on it. See svdq_gemm_qnext.cuh for why a low-rank next layer is
+// not fused.
+bool qnext_fused(const svdq_shape& s, int next_rank) {
+  return next_rank == 0 && gemm_choice(s) == 256 && pair_clusters<256, true>() > 0;
+}
+
+size_t qnext_workspace_bytes(const svdq_shape& s, int next_rank) {
+  return qnext_fused(s, next_rank) ? 0 : (size_t)s.M * (size_t)s.N * 2u;
 }
 
 template <int RANK>
@@ -717,6 +739,58 @@ svdq_status svdq_linear(svdq_shape s, const void* Qx, const void* Sx, const void
   if ((r = launch_gemm(s, 0, Qx, Sx, nullptr, Qr, Sr, nullptr, Y, st)) != SVDQ_OK) return r;
   if (s.rank == 0) return SVDQ_OK;
   return launch_up_rmw(s, s.rank, T, L2t, Y, st);
+}
+
+svdq_status svdq_linear_quantize_next_workspace(svdq_shape s, int32_t next_rank, size_t* bytes) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (next_rank < 0 || next_rank > 128 || next_rank % 16)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "next rank %d: need one of 0, 16, ..., 128", (int)next_rank);
+  if (!bytes) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  if (s.M == 0) {
+    *bytes = 0;
+    return SVDQ_OK;
+  }
+  if ((r = check_device()) != SVDQ_OK) return r;
+  *bytes = qnext_workspace_bytes(s, next_rank);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_linear_quantize_next(svdq_shape s, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                                      const void* Sr, const void* L2t, int32_t next_rank,
+                                      const float* next_inv_lambda, const void* next_L1p, void* next_Qx,
+                                      void* next_Sx, void* next_T, void* Y, void* workspace, size_t workspace_bytes,
+                                      void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  const svdq_shape ns = {s.M, s.N, 128, next_rank};   // the next layer reads Y as its X (K' = N)
+  if ((r = check_shape(ns)) != SVDQ_OK) return r;
+  if (s.M == 0) return SVDQ_OK;
+  if (!Qx || !Sx || !Qr || !Sr || (s.rank > 0 && (!T || !L2t)) || !next_inv_lambda || !next_Qx || !next_Sx ||
+      (next_rank > 0 && (!next_L1p || !next_T)))
+    return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {Qx, Sx, T, Qr, Sr, L2t, next_inv_lambda, next_L1p, next_Qx, next_Sx, next_T, Y, workspace};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  const bool fused = qnext_fused(s, next_rank);
+  const size_t need = Y ? 0 : qnext_workspace_bytes(s, next_rank);
+  if (need > 0 && (workspace_bytes < need || !workspace))
+    return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "workspace of %zu bytes needed", need);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!fused) {   // Y (into the workspace unless the caller wants it), then the quantizer
+    void* y = Y ? Y : workspace;
+    if ((r = launch_gemm(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, y, st)) != SVDQ_OK) return r;
+    return launch_quant<true>(ns, next_rank, y, next_inv_lambda, next_L1p, next_Qx, next_Sx, next_T, st);
+  }
+  svdq::NextQuant nq;
+  nq.inv_lambda = next_inv_lambda;
+  nq.qx = static_cast<uint8_t*>(next_Qx);
+  nq.sx = static_cast<uint8_t*>(next_Sx);
+  return launch_gemm_pair<256, true>(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<256, true>(), nq,
+                                     Y != nullptr);
 }
 
 namespace svdq {

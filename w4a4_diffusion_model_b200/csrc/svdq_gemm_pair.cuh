@@ -35,6 +35,7 @@
 #include <cuda_bf16.h>
 
 #include "svdq_gemm_common.cuh"
+#include "svdq_gemm_qnext.cuh"
 #include "svdq_ptx.cuh"
 
 namespace svdq {
@@ -69,12 +70,15 @@ struct PairCfg {
 // tm_qr / tm_l2 boxes are 128 rows (NB = 256) or 64 rows (NB = 384).
 // tm_sfa / tm_sfb view a native scale buffer as 3-D uint8
 // [row blocks][K/64 * 2 chunks][256 bytes]; box {256, 8, 1 | NB/128} (4 atoms per row block).
-template <int NB>
+// QNEXT: the epilogue also quantizes Y for the next layer (svdq_gemm_qnext.cuh),
+// and stores Y itself only when store_y is set.
+template <int NB, bool QNEXT = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     const __grid_constant__ CUtensorMap tm_qx, const __grid_constant__ CUtensorMap tm_qr,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
-    const __grid_constant__ CUtensorMap tm_y, int M, int N, int K, int rank) {
+    const __grid_constant__ CUtensorMap tm_y, int M, int N, int K, int rank, NextQuant nq, int store_y) {
+  static_assert(!QNEXT || NB == 256, "the next layer's quantization runs on 256 x 256 tiles");
   using C = PairCfg<NB>;
   constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -107,6 +111,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     mbar_init(acc_empty, 2 * kGemmEpiWarps);
     mbar_init(mma_drain, 1);
     fence_mbar_init();
+  }
+  __shared__ float rcp_tbl[QNEXT ? 128 : 1];   // fp32(1/s) per E4M3 byte with the sign bit clear
+  if (QNEXT && threadIdx.x < 128) {
+    const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)threadIdx.x, __NV_E4M3)));
+    rcp_tbl[threadIdx.x] = __frcp_rn(sv);
   }
   if (warp == kMmaWarp) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
@@ -307,7 +316,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     const int q = warp & 3, h = warp >> 2;
     unsigned char* box = smem + C::kEpiOffset + warp * kEpiBoxBytes;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
-    if (lane == 0) prefetch_tmap(&tm_y);
+    if (lane == 0 && (!QNEXT || store_y)) prefetch_tmap(&tm_y);
     uint32_t tcount = 0;
     for (int tile = cluster; tile < ntiles; tile += nclusters, ++tcount) {
       const int m0 = (tile / tiles_n) * kPairBM + 128 * (int)crank;
@@ -324,7 +333,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // this warp's part of the accumulator is drained
-        epilogue_store_band<2>(p, box, &tm_y, n0 + h * 128, m0 + 32 * q, lane, store);
+        if (QNEXT)
+          epilogue_quantize_next<2>(p, box, nq, rcp_tbl, &tm_y, store_y != 0, m0 + 32 * q, n0 + h * 128, M, N, lane);
+        else
+          epilogue_store_band<2>(p, box, &tm_y, n0 + h * 128, m0 + 32 * q, lane, store);
       } else {   // drain all 192 columns before releasing the accumulator, then store
         uint32_t p2[32];
         epilogue_drain_pack<2>(taddr + 128, p2);

@@ -30,7 +30,8 @@ STATUS = {
 EXPORTS = [
     "svdq_status_string", "svdq_last_error", "svdq_version", "svdq_act_sizes", "svdq_weight_sizes",
     "svdq_channel_amax", "svdq_prepare_weights", "svdq_prepare_weights_static", "svdq_quantize_act",
-    "svdq_linear", "svdq_append_lowrank", "svdq_selftest_timeout", "svdq_scales_to_canonical", "svdq_check",
+    "svdq_linear", "svdq_linear_quantize_next", "svdq_linear_quantize_next_workspace", "svdq_append_lowrank",
+    "svdq_selftest_timeout", "svdq_scales_to_canonical", "svdq_check",
 ]
 
 
@@ -80,6 +81,11 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_linear.restype = st
     lib.svdq_scales_to_canonical.argtypes, lib.svdq_scales_to_canonical.restype = [i64, i64, vp, vp, vp], st
     lib.svdq_check.argtypes, lib.svdq_check.restype = [vp], st
+    lib.svdq_linear_quantize_next.argtypes = [Shape, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp,
+                                              vp, sz, vp]
+    lib.svdq_linear_quantize_next.restype = st
+    lib.svdq_linear_quantize_next_workspace.argtypes = [Shape, ctypes.c_int32, P(sz)]
+    lib.svdq_linear_quantize_next_workspace.restype = st
     _lib = lib
     return lib
 
@@ -195,6 +201,39 @@ def svdq_linear(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: P
     _check(load().svdq_linear(shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t), _ptr(Y),
                               variant, _stream()))
     return Y
+
+
+def svdq_linear_quantize_next_workspace(shape: LayerShape, next_rank: int) -> int:
+    v = ctypes.c_size_t()
+    _check(load().svdq_linear_quantize_next_workspace(shape.c(), next_rank, ctypes.byref(v)))
+    return v.value
+
+
+def svdq_linear_quantize_next(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: PreparedWeights,
+                              next_inv_lambda: torch.Tensor, next_L1p: torch.Tensor | None, next_rank: int,
+                              store_y: bool = False, out: tuple | None = None, workspace: torch.Tensor | None = None):
+    """svdq_linear whose epilogue also quantizes Y for the next layer (K' = N).
+    Returns (next_Qx [M][N/2] uint8, next_Sx native uint8, next_T [M][next_rank] bf16 or None,
+    Y [M][N] bf16 or None)."""
+    M = Qx.shape[0]
+    K, N, rank = W.shape.K, W.shape.N, W.shape.rank
+    shape = LayerShape(M, K, N, rank)
+    dev = Qx.device
+    if out is None:
+        _, sxb, _ = svdq_act_sizes(LayerShape(M, N, 128, next_rank))
+        Qn = torch.empty(M, N // 2, dtype=torch.uint8, device=dev)
+        Sn = torch.empty(sxb, dtype=torch.uint8, device=dev)
+        Tn = torch.empty(M, next_rank, dtype=torch.bfloat16, device=dev) if next_rank else None
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if store_y else None
+    else:
+        Qn, Sn, Tn, Y = out
+    need = svdq_linear_quantize_next_workspace(shape, next_rank)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(load().svdq_linear_quantize_next(
+        shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t), next_rank, _ptr(next_inv_lambda),
+        _ptr(next_L1p), _ptr(Qn), _ptr(Sn), _ptr(Tn), _ptr(Y), _ptr(workspace), workspace.numel(), _stream()))
+    return Qn, Sn, Tn, Y
 
 
 def svdq_scales_to_canonical(native: torch.Tensor, rows: int, K: int) -> torch.Tensor:
