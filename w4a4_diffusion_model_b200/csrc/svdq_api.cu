@@ -227,17 +227,19 @@ struct QuantLaunch {
                                    64, RANK, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
       return r;
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = ksplit;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = ksplit;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.gridDim = dim3(rowblocks * ksplit, 1, 1);
     cfg.blockDim = dim3(L::kThreads, 1, 1);
     cfg.dynamicSmemBytes = L::kBytes;
     cfg.stream = st;
     cfg.attrs = attr;
-    cfg.numAttrs = (RANK > 0 && ksplit > 1) ? 1 : 0;
+    cfg.numAttrs = (RANK > 0 && ksplit > 1) ? 2 : 1;
     SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tx, tl, inv, static_cast<uint8_t*>(Qx), static_cast<uint8_t*>(Sx),
                                  static_cast<__nv_bfloat16*>(T), (int)s.M, (int)s.K, ksplit));
     return SVDQ_OK;
@@ -305,26 +307,40 @@ svdq_status launch_gemm_single(const svdq_shape& s, int rank, const void* Qx, co
   SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
   const long long tiles = ((s.M + svdq::kGemmBM - 1) / svdq::kGemmBM) * ((s.N + svdq::kGemmBN - 1) / svdq::kGemmBN);
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, svdq::kGemmThreads, L::kBytes, st>>>(tqx, tqr, tt, tl, ty, static_cast<const uint8_t*>(Sx),
-                                                   static_cast<const uint8_t*>(Sr), (int)s.M, (int)s.N, (int)s.K,
-                                                   rank);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
+  cfg.dynamicSmemBytes = L::kBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tt, tl, ty, static_cast<const uint8_t*>(Sx),
+                               static_cast<const uint8_t*>(Sr), (int)s.M, (int)s.N, (int)s.K, rank));
   SVDQ_LAUNCHED("svdq_gemm_kernel");
   return SVDQ_OK;
 }
 
+// Launch configuration of the pair kernel: clusters of 2 CTAs, and (for real
+// launches) programmatic stream serialization, so that the kernel's prologue
+// overlaps the end of the previous kernel of the stream. `attr` must hold 2.
 template <int NB>
-cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr) {
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr, bool pdl = true) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
   cfg.dynamicSmemBytes = svdq::PairCfg<NB>::kBytes;
   cfg.stream = st;
-  attr->id = cudaLaunchAttributeClusterDimension;
-  attr->val.clusterDim.x = 2;
-  attr->val.clusterDim.y = 1;
-  attr->val.clusterDim.z = 1;
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   return cfg;
 }
 
@@ -342,8 +358,8 @@ int pair_clusters() {
     cudaGetLastError();
     return 0;
   }
-  cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, &attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, attr, false);
   int n = 0;
   if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
     cudaGetLastError();
@@ -389,8 +405,8 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
   auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
   const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / NB);
   const int ncl = (int)(tiles < clusters ? tiles : clusters);
-  cudaLaunchAttribute attr;
-  cudaLaunchConfig_t cfg = pair_config<NB>(ncl, st, &attr);
+  cudaLaunchAttribute attr[2];
+  cudaLaunchConfig_t cfg = pair_config<NB>(ncl, st, attr);
   SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank, nq,
                                store_y ? 1 : 0));
   SVDQ_LAUNCHED("svdq_gemm_pair_kernel");

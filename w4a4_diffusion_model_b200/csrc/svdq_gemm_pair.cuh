@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated in both
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dependency_wait();     // the previous kernel's outputs (Qx, Sx, T) are complete
+  grid_launch_dependents();
 
   if (warp == kProducerWarp) {
     if (lane == 0) {

@@ -44,6 +44,23 @@ __device__ __forceinline__ bool device_error_set() {
   return *((volatile unsigned int*)&g_device_error) != 0u;
 }
 
+// ---------------------------------------------------------------- dependent launch
+// Kernels launched with programmatic stream serialization run their prologue
+// (barrier set-up, TMEM allocation, descriptor prefetch) while the previous
+// kernel of the stream finishes, then wait here for it to complete (and its
+// memory to be visible) before touching global memory. Without that launch
+// attribute the wait returns at once.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel of the stream be scheduled once every CTA of this grid
+// has called this or exited; its CTAs then occupy SMs as this grid's CTAs leave
+// them and wait in grid_dependency_wait(). Every CTA of this grid is already
+// resident when the last one calls it, so the next grid cannot take an SM that
+// this one still needs.
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

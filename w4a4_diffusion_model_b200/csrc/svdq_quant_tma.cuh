@@ -168,6 +168,8 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = RANK > 0 ? *tmem_slot : 0u;
+  grid_dependency_wait();     // the previous kernel is complete (it may still read Qx, Sx, T or write X)
+  grid_launch_dependents();
 
   if (warp == L::kProducerWarp) {
     // ------------------------------------------------------------------ producer
