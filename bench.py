@@ -544,23 +544,67 @@ def run_ours(args):
         extras["lowrank_overhead_gemm"] = round(statistics.mean(k2f) / extras["rank0_gemm_ms"] - 1, 4)
         extras["unfused_overhead_layer"] = round(extras["unfused_layer_ms"] / extras["rank0_layer_ms"] - 1, 4)
 
-        # end to end through the public API with host buffers: pinned X in, Y out
+        # end to end through the public API with host buffers: every step copies
+        # its X in from pinned host memory and its Y out to pinned host memory.
         X_host = X_cpu.pin_memory()
-        Y_host = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+        Y_host = [torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
 
-        def e2e_step(i, ev):
+        def e2e_step(i, ev):       # one step at a time: upload, layer, download
             ev[0].record(stream)
             X.copy_(X_host, non_blocking=True)
             S.svdq_quantize_act(X, P.inv_lam, P.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
             S.svdq_linear(Qx, Sx, T, P, S.SVDQ_FUSED, out=Y)
-            Y_host.copy_(Y, non_blocking=True)
+            Y_host[0].copy_(Y, non_blocking=True)
             ev[1].record(stream)
             ev[2].record(stream)
         ke, _ = timed(n_x, e2e_step)
-        e2e_ms = aggregate_max(sum(ke), world) / n_x
+        e2e_serial_ms = aggregate_max(sum(ke), world) / n_x
+
+        # the same, pipelined as a serving loop would run it: uploads and
+        # downloads on their own streams (one copy engine per direction), two
+        # device buffer sets, so step i's layer overlaps step i+1's upload and
+        # step i-1's download; the timed region spans the first upload to the
+        # last download
+        Xd, Yd = [X, X.clone()], [Y, torch.empty_like(Y)]
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        up, done, down = ([torch.cuda.Event() for _ in range(2)] for _ in range(3))
+
+        def e2e_pipelined(n):
+            t_a, t_b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            torch.cuda._sleep(2_000_000)
+            t_a.record(stream)
+            s_in.wait_stream(stream)
+            s_out.wait_stream(stream)
+            for i in range(n):
+                b = i % 2
+                if i >= 2:
+                    s_in.wait_event(done[b])          # step i-2's layer has read Xd[b]
+                with torch.cuda.stream(s_in):
+                    Xd[b].copy_(X_host, non_blocking=True)
+                up[b].record(s_in)
+                stream.wait_event(up[b])
+                if i >= 2:
+                    stream.wait_event(down[b])        # step i-2's Y has left Yd[b]
+                S.svdq_quantize_act(Xd[b], P.inv_lam, P.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
+                S.svdq_linear(Qx, Sx, T, P, S.SVDQ_FUSED, out=Yd[b])
+                done[b].record(stream)
+                s_out.wait_event(done[b])
+                with torch.cuda.stream(s_out):
+                    Y_host[b].copy_(Yd[b], non_blocking=True)
+                down[b].record(s_out)
+            stream.wait_stream(s_in)
+            stream.wait_stream(s_out)
+            t_b.record(stream)
+            torch.cuda.synchronize()
+            return t_a.elapsed_time(t_b)
+        e2e_pipelined(3)
+        e2e_ms = aggregate_max(e2e_pipelined(n_x), world) / n_x
         e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
-               "ms_per_step": round(e2e_ms, 4)}
+               "ms_per_step": round(e2e_ms, 4),
+               "pipeline": "uploads and downloads on their own streams, two device buffer sets",
+               "ms_per_step_one_at_a_time": round(e2e_serial_ms, 4)}
         S.svdq_check()
 
         if rank_id == 0 and world == 1:
