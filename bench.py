@@ -520,6 +520,11 @@ def run_ours(args):
         kc, _ = timed(n_x, cublas)
         # warm L2: the same inputs every step (no rotation)
         k1w, k2w = timed(n_x, lambda i, ev: step(0, ev=ev))
+        # the GEMM alone, launched back to back on the rotating inputs with one
+        # pair of events around the block: its sustained duration per launch
+        # (the per-kernel pass above also pays each launch's latency)
+        gemm_block_ms = timed_block(n_x, lambda i: S.svdq_linear(Qx, Sx, T if w.rank else None, sets[i % n_sets][1],
+                                                                  S.SVDQ_FUSED, out=Y)) / n_x
         lay = statistics.mean(step_ms)
         lay_f = statistics.mean(a + b for a, b in zip(k1f, k2f))
         q10, q50, q90 = np.percentile(step_ms, [10, 50, 90])
@@ -535,6 +540,8 @@ def run_ours(args):
             "unfused_layer_ms": round(statistics.mean(a + b for a, b in zip(k1u, k2u)), 4),
             "rank0_layer_ms": round(statistics.mean(a + b for a, b in zip(k1z, k2z)), 4),
             "rank0_gemm_ms": round(statistics.mean(k2z), 4),
+            "gemm_block_ms": round(gemm_block_ms, 4),
+            "gemm_block_frac": round(gemm_flops(w) / (gemm_block_ms * 1e-3) / 1e12 / fp4_peak, 4),
             "bf16_cublas_ms": round(statistics.mean(kc), 4),
             "bf16_cublas_tflops": round(2 * w.M * w.N * w.K / (statistics.mean(kc) * 1e-3) / 1e12, 1),
         }
