@@ -551,6 +551,47 @@ def run_ours(args):
         extras["lowrank_overhead_gemm"] = round(statistics.mean(k2f) / extras["rank0_gemm_ms"] - 1, 4)
         extras["unfused_overhead_layer"] = round(extras["unfused_layer_ms"] / extras["rank0_layer_ms"] - 1, 4)
 
+        # the INT4 variant (64-element groups, fp16 scales) of the same layer:
+        # same smoothing and low-rank factors, INT4 residual and activation
+        sets4 = [S.svdq_int4_prepare_weights(W, P_) for _, P_, _ in sets]
+        Qx4 = torch.empty(w.M, w.K, dtype=torch.uint8, device=dev)
+        Sx4 = torch.empty(w.K // 64, (w.M + 127) // 128 * 128, dtype=torch.float32, device=dev)
+
+        def step4(i, ev=None):
+            X_, P_, _ = sets[i % n_sets]
+            if ev is not None:
+                ev[0].record(stream)
+            S.svdq_int4_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, out=(Qx4, Sx4, T))
+            if ev is not None:
+                ev[1].record(stream)
+            S.svdq_int4_linear(Qx4, Sx4, T, sets4[i % n_sets], out=Y)
+            if ev is not None:
+                ev[2].record(stream)
+        for i in range(3):
+            step4(i)
+        int4_layer = timed_block(n_x, lambda i: step4(i)) / n_x
+        k1i, k2i = timed(n_x, lambda i, ev: step4(i, ev), warm=0)
+        int4_gemm_block = timed_block(n_x, lambda i: S.svdq_int4_linear(Qx4, Sx4, T, sets4[i % n_sets], out=Y)) / n_x
+        S.svdq_check()
+        g4 = statistics.mean(k2i)
+        sm_hz = ((clocks or {}).get("sm_mhz") or 1900) * 1e6
+        # the rescale bound: two fp32 operations per output element and 64-group
+        # (128 GEMM flops), 128 fp32 lanes per SM
+        alu_peak = 64 * 128 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz / 1e12
+        fp8_peak = 2 * peaks["bf16_tflops_sustained"]
+        extras["int4"] = {
+            "layer_ms": round(int4_layer, 4),
+            "layer_tflops": round(flops_step / (int4_layer * 1e-3) / 1e12, 1),
+            "quantize_ms": round(statistics.mean(k1i), 4),
+            "gemm_ms": round(g4, 4),
+            "gemm_tflops": round(gemm_flops(w) / (g4 * 1e-3) / 1e12, 1),
+            "gemm_block_ms": round(int4_gemm_block, 4),
+            "gemm_block_tflops": round(gemm_flops(w) / (int4_gemm_block * 1e-3) / 1e12, 1),
+            "gemm_block_frac_alu": round(gemm_flops(w) / (int4_gemm_block * 1e-3) / 1e12 / alu_peak, 4),
+            "gemm_block_frac_fp8": round(gemm_flops(w) / (int4_gemm_block * 1e-3) / 1e12 / fp8_peak, 4),
+            "alu_peak_tflops": round(alu_peak, 1), "fp8_peak_tflops": round(fp8_peak, 1),
+        }
+
         # end to end through the public API with host buffers: every step copies
         # its X in from pinned host memory and its Y out to pinned host memory.
         X_host = X_cpu.pin_memory()

@@ -234,6 +234,55 @@ SVDQ_API svdq_status svdq_append_lowrank(svdq_shape shape, int32_t extra, const 
                                          const void* A, const void* B, void* L1p_out, void* L2t_out,
                                          void* stream);
 
+/* ---------------------------------------------------------------- INT4 variant
+ * The same layer with INT4 in place of NVFP4 (the pages' path for GPUs without
+ * FP4 tensor cores: walkthrough eq. (1) with q_max = 2^(4-1) - 1 = 7; handbook,
+ * Quantization chapter: one fp16 scale per 64 elements). Per 64-element group
+ * along K:  s = fp16_rne(min(fp32(max|v| / 7), 65504)),
+ *           q = clamp(rint(fp32(v * fp32(1/s))), -7, 7)  (all 0 when s == 0),
+ * and Y = bf16( sum_g sx[m,g] sw[n,g] sum_{k in g} qx[m,k] qr[n,k] + T L2 ).
+ * Smoothing, L1p, L2t and T are those of the NVFP4 layer (svdq_prepare_weights);
+ * only the residual and the activation are encoded differently.
+ *
+ * Buffer formats (sizes from svdq_int4_act_sizes / svdq_int4_weight_sizes):
+ *   int4 codes   uint8 [rows][K]: one byte per code, the E4M3 encoding of the
+ *                integer (0x00 for 0, 0x38 for 1, ..., 0x4E for 7, sign bit 0x80
+ *                for negatives). sm_100a has no 4-bit integer MMA; E4M3 holds
+ *                every code exactly and feeds the FP8 tensor cores, at twice
+ *                the bytes of packed nibbles.
+ *   int4 scales  fp32 [K/64][rows_pad], group-major: scale of (row r, group g)
+ *                at g * rows_pad + r. Every value is an fp16 value. rows_pad =
+ *                ceil(M/128)*128 for the activation (rows past M hold 0) and N for
+ *                the weight.
+ * Shapes as for the NVFP4 entry points. */
+SVDQ_API svdq_status svdq_int4_act_sizes(svdq_shape shape, size_t* qx, size_t* sx, size_t* t);
+SVDQ_API svdq_status svdq_int4_weight_sizes(svdq_shape shape, size_t* qr, size_t* sr);
+
+/* INT4 codes and scales of the residual R = W_hat - (lambda L1p^T) L2 (eq. (5);
+ * fp64 with every product exact, rounded to fp32 once, exactly as
+ * svdq_prepare_weights forms it), grouped along K for every output channel.
+ * W_lin bf16 [N][K], lambda fp32 [K], L1p bf16 [rank][K], L2t bf16 [N][rank]
+ * as written by svdq_prepare_weights (L1p and L2t may be NULL when rank == 0).
+ * Writes Qr uint8 [N][K] and Sr fp32 [K/64][N]. Stream-ordered. */
+SVDQ_API svdq_status svdq_int4_quantize_residual(svdq_shape shape, const void* W_lin, const float* lambda,
+                                                 const void* L1p, const void* L2t, void* Qr, void* Sr, void* stream);
+
+/* Hot path, step 1 (INT4): one read of X bf16 [M][K] -> smoothing, INT4 codes
+ * Qx uint8 [M][K] and scales Sx fp32 [K/64][ceil(M/128)*128], and the fused
+ * down-projection T bf16 [M][rank] = bf16(X L1p^T) (same kernel as
+ * svdq_quantize_act, INT4 encoder). Async on stream. */
+SVDQ_API svdq_status svdq_int4_quantize_act(svdq_shape shape, const void* X, const float* inv_lambda,
+                                            const void* L1p, void* Qx, void* Sx, void* T, void* stream);
+
+/* Hot path, step 2 (INT4): Y bf16 [M][N]. Each group's integer products run on
+ * FP8 tensor cores into fp32 tensor memory (exact); the group's scale product
+ * fp32(sx * sw) (exact) is applied with one fused multiply-add per element into
+ * fp32 accumulators; T L2 is added from a bf16 MMA; Y = bf16_rne of the sum.
+ * Qx/Sx from svdq_int4_quantize_act, Qr/Sr from svdq_int4_quantize_residual,
+ * T and L2t as for svdq_linear (NULL allowed when rank == 0). Async on stream. */
+SVDQ_API svdq_status svdq_int4_linear(svdq_shape shape, const void* Qx, const void* Sx, const void* T,
+                                      const void* Qr, const void* Sr, const void* L2t, void* Y, void* stream);
+
 /* Diagnostic of the failure path (the pages have no counterpart): one thread
  * waits, with the library's bounded wait, on a barrier phase that nothing
  * completes; after the wait limit (2 s) it records the device error word and

@@ -83,3 +83,15 @@ def test_int4_layer_error_trends():
     ef_r16 = O.rel_fro(O.layer_reference(Xn, Wn, 0.5, 16)["Y"], exact)
     assert e4_r16 < e4_r0 < 0.5
     assert ef_r16 < e4_r16 < 4 * ef_r16
+
+
+def test_int4_codes_as_e4m3_bytes_match_torch():
+    """The byte form of INT4 codes used by the B200 kernels: the E4M3 encoding
+    of the integers -7..7 is exact, and the oracle's encoder (with the sign bit)
+    agrees with torch's float8_e4m3fn conversion."""
+    import torch
+    ints = np.arange(-7, 8)
+    ours = (O.e4m3_encode(np.abs(ints).astype(np.float64)) | np.where(ints < 0, 0x80, 0)).astype(np.uint8)
+    lib = torch.tensor(ints, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(ours, lib)
+    assert np.array_equal(O.e4m3_decode(ours), ints.astype(np.float64))

@@ -13,6 +13,7 @@
 #include "svdq.h"
 #include "svdq_gemm.cuh"
 #include "svdq_gemm_pair.cuh"
+#include "svdq_int4.cuh"
 #include "svdq_prepare.cuh"
 #include "svdq_quant.cuh"
 #include "svdq_quant_tma.cuh"
@@ -157,10 +158,10 @@ int sm_count() {
 // last scale atom get zero scales. With a low-rank branch the K slices of a
 // row block form a cluster (their partial T is summed through distributed
 // shared memory) and all clusters must be resident at once.
-template <int RANK, int BM, bool QUANT>
+template <int RANK, int BM, int CODEC>
 struct QuantLaunch {
   using L = svdq::QuantSmem<RANK, BM>;
-  static constexpr auto kern = svdq::quantize_tma_kernel<RANK, BM, QUANT>;
+  static constexpr auto kern = svdq::quantize_tma_kernel<RANK, BM, CODEC>;
 
   static svdq_status prepare() {   // once per device
     static bool done[64];
@@ -247,11 +248,11 @@ struct QuantLaunch {
 };
 
 // 128-row CTAs unless 64-row CTAs put more of them in the one wave.
-template <int RANK, bool QUANT>
+template <int RANK, int CODEC>
 svdq_status launch_quant_t(const svdq_shape& s, const void* X, const float* inv, const void* L1p, void* Qx, void* Sx,
                            void* T, cudaStream_t st) {
-  using Big = QuantLaunch<RANK, 128, QUANT>;
-  using Small = QuantLaunch<RANK, 64, QUANT>;
+  using Big = QuantLaunch<RANK, 128, CODEC>;
+  using Small = QuantLaunch<RANK, 64, CODEC>;
   if (s.M == 0) return SVDQ_OK;
   svdq_status r;
   if ((r = Big::prepare()) != SVDQ_OK || (r = Small::prepare()) != SVDQ_OK) return r;
@@ -261,13 +262,13 @@ svdq_status launch_quant_t(const svdq_shape& s, const void* X, const float* inv,
   return Big::launch(s, kb, X, inv, L1p, Qx, Sx, T, st);
 }
 
-template <bool QUANT>
+template <int CODEC>
 svdq_status launch_quant(const svdq_shape& s, int rank, const void* X, const float* inv, const void* L1p, void* Qx,
                          void* Sx, void* T, cudaStream_t st) {
   switch (rank) {
 #define SVDQ_CASE(R) \
   case R:            \
-    return launch_quant_t<R, QUANT>(s, X, inv, L1p, Qx, Sx, T, st);
+    return launch_quant_t<R, CODEC>(s, X, inv, L1p, Qx, Sx, T, st);
     SVDQ_CASE(0) SVDQ_CASE(16) SVDQ_CASE(32) SVDQ_CASE(48) SVDQ_CASE(64) SVDQ_CASE(80) SVDQ_CASE(96)
     SVDQ_CASE(112) SVDQ_CASE(128)
 #undef SVDQ_CASE
@@ -591,6 +592,51 @@ svdq_status launch_channel_amax(int64_t rows, int64_t K, const void* X, float* a
   return SVDQ_OK;
 }
 
+// ---------------------------------------------------------------- INT4 variant
+size_t int4_act_scale_bytes(int64_t M, int64_t K) { return (size_t)(K / 64) * (size_t)((M + 127) / 128 * 128) * 4u; }
+
+svdq_status launch_int4_gemm(const svdq_shape& s, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                             const void* Sr, const void* L2t, void* Y, cudaStream_t st) {
+  CUtensorMap tqx, tqr, tt, tl;
+  svdq_status r;
+  if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K, (uint64_t)s.M, svdq::kI4KTile,
+                     svdq::kI4BM, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if ((r = make_tmap(&tqr, Qr, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K, (uint64_t)s.N, svdq::kI4KTile,
+                     svdq::kI4BN, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+    return r;
+  if (s.rank > 0) {
+    if ((r = make_tmap(&tt, T, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.rank, (uint64_t)s.M, svdq::kGemmLrK,
+                       svdq::kI4BM, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+    if ((r = make_tmap(&tl, L2t, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.rank, (uint64_t)s.N,
+                       svdq::kGemmLrK, svdq::kI4BN, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+  } else {
+    memset(&tt, 0, sizeof(tt));
+    memset(&tl, 0, sizeof(tl));
+  }
+  auto kern = svdq::svdq_int4_gemm_kernel;
+  SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::kI4SmemBytes));
+  const long long tiles = ((s.M + svdq::kI4BM - 1) / svdq::kI4BM) * ((s.N + svdq::kI4BN - 1) / svdq::kI4BN);
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(svdq::kI4Threads, 1, 1);
+  cfg.dynamicSmemBytes = svdq::kI4SmemBytes;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tt, tl, static_cast<const float*>(Sx),
+                               static_cast<const float*>(Sr), static_cast<__nv_bfloat16*>(Y), (int)s.M, (int)s.N,
+                               (int)s.K, (int)s.rank));
+  SVDQ_LAUNCHED("svdq_int4_gemm_kernel");
+  return SVDQ_OK;
+}
+
 }  // namespace
 
 // ============================================================================ C ABI
@@ -732,10 +778,10 @@ svdq_status svdq_quantize_act(svdq_shape s, const void* X, const float* inv_lamb
     if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
   if ((r = check_device()) != SVDQ_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (variant == SVDQ_FUSED) return launch_quant<true>(s, s.rank, X, inv_lambda, L1p, Qx, Sx, T, st);
-  if ((r = launch_quant<true>(s, 0, X, inv_lambda, nullptr, Qx, Sx, nullptr, st)) != SVDQ_OK) return r;
+  if (variant == SVDQ_FUSED) return launch_quant<svdq::kCodecNvfp4>(s, s.rank, X, inv_lambda, L1p, Qx, Sx, T, st);
+  if ((r = launch_quant<svdq::kCodecNvfp4>(s, 0, X, inv_lambda, nullptr, Qx, Sx, nullptr, st)) != SVDQ_OK) return r;
   if (s.rank == 0) return SVDQ_OK;
-  return launch_quant<false>(s, s.rank, X, nullptr, L1p, nullptr, nullptr, T, st);
+  return launch_quant<svdq::kCodecNone>(s, s.rank, X, nullptr, L1p, nullptr, nullptr, T, st);
 }
 
 svdq_status svdq_linear(svdq_shape s, const void* Qx, const void* Sx, const void* T, const void* Qr, const void* Sr,
@@ -799,7 +845,7 @@ svdq_status svdq_linear_quantize_next(svdq_shape s, const void* Qx, const void* 
   if (!fused) {   // Y (into the workspace unless the caller wants it), then the quantizer
     void* y = Y ? Y : workspace;
     if ((r = launch_gemm(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, y, st)) != SVDQ_OK) return r;
-    return launch_quant<true>(ns, next_rank, y, next_inv_lambda, next_L1p, next_Qx, next_Sx, next_T, st);
+    return launch_quant<svdq::kCodecNvfp4>(ns, next_rank, y, next_inv_lambda, next_L1p, next_Qx, next_Sx, next_T, st);
   }
   svdq::NextQuant nq;
   nq.inv_lambda = next_inv_lambda;
@@ -860,6 +906,71 @@ svdq_status svdq_append_lowrank(svdq_shape s, int32_t extra, const void* L1p, co
                                                 static_cast<uint4*>(L2t_out), (int)s.N, (int)s.rank, (int)extra);
   SVDQ_LAUNCHED("append_l2t_kernel");
   return SVDQ_OK;
+}
+
+svdq_status svdq_int4_act_sizes(svdq_shape s, size_t* qx, size_t* sx, size_t* t) {
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (qx) *qx = (size_t)s.M * (size_t)s.K;
+  if (sx) *sx = int4_act_scale_bytes(s.M, s.K);
+  if (t) *t = (size_t)s.M * (size_t)s.rank * 2u;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_int4_weight_sizes(svdq_shape s, size_t* qr, size_t* sr) {
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (qr) *qr = (size_t)s.N * (size_t)s.K;
+  if (sr) *sr = (size_t)(s.K / 64) * (size_t)s.N * 4u;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_int4_quantize_residual(svdq_shape s, const void* W, const float* lambda, const void* L1p,
+                                        const void* L2t, void* Qr, void* Sr, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (!W || !lambda || !Qr || !Sr || (s.rank > 0 && (!L1p || !L2t))) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {W, lambda, L1p, L2t, Qr, Sr};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  const long long n_threads = s.N * (s.K / 16);
+  svdq::residual_quantize_int4_kernel<<<(unsigned)((n_threads + 127) / 128), 128, 0,
+                                        static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const __nv_bfloat16*>(W), lambda, static_cast<const __nv_bfloat16*>(L1p),
+      static_cast<const __nv_bfloat16*>(L2t), static_cast<uint8_t*>(Qr), static_cast<float*>(Sr), (int)s.N, (int)s.K,
+      (int)s.rank);
+  SVDQ_LAUNCHED("residual_quantize_int4_kernel");
+  return SVDQ_OK;
+}
+
+svdq_status svdq_int4_quantize_act(svdq_shape s, const void* X, const float* inv_lambda, const void* L1p, void* Qx,
+                                   void* Sx, void* T, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (s.M == 0) return SVDQ_OK;
+  if (!X || !inv_lambda || !Qx || !Sx || (s.rank > 0 && (!L1p || !T))) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {X, inv_lambda, Qx, Sx, L1p, T};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  return launch_quant<svdq::kCodecInt4>(s, s.rank, X, inv_lambda, L1p, Qx, Sx, T, static_cast<cudaStream_t>(stream));
+}
+
+svdq_status svdq_int4_linear(svdq_shape s, const void* Qx, const void* Sx, const void* T, const void* Qr,
+                             const void* Sr, const void* L2t, void* Y, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_shape(s);
+  if (r != SVDQ_OK) return r;
+  if (s.M == 0) return SVDQ_OK;
+  if (!Qx || !Sx || !Qr || !Sr || !Y || (s.rank > 0 && (!T || !L2t))) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {Qx, Sx, T, Qr, Sr, L2t, Y};
+  for (const void* p : ptrs)
+    if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  return launch_int4_gemm(s, Qx, Sx, T, Qr, Sr, L2t, Y, static_cast<cudaStream_t>(stream));
 }
 
 svdq_status svdq_selftest_timeout(void* stream) {

@@ -11,7 +11,8 @@
 // Quantization: 16 warps own 16 rows and one 64-column slab of every stage
 // each (with RG = BM/16 row groups, warp w takes rows 16 (w mod RG) + [0, 16)
 // and slab w / RG). Thread (g = lane/4, t = lane%4) quantizes rows g and g+8,
-// columns [16t, 16t+16) of the slab -- one quantization group per row.
+// columns [16t, 16t+16) of the slab: one NVFP4 group per row, or a quarter of
+// an INT4 group (64 elements; the four threads of a quad share it).
 //
 // Down-projection: one thread issues tcgen05 kind::f16 MMAs on the same
 // shared-memory tiles (X box as A, L1p box as B, both K-major with 128B
@@ -28,6 +29,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_fp4.h>
 #include <cuda_fp8.h>
 
@@ -126,11 +128,65 @@ __device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float
   codes = b != 0u ? make_uint2(lo, hi) : make_uint2(0u, 0u);
 }
 
-template <int RANK, int BM, bool QUANT>
+// What the quantizing warps produce besides T.
+enum QuantCodec : int {
+  kCodecNone = 0,    // T only (the unfused variant's second pass)
+  kCodecNvfp4 = 1,   // packed E2M1 codes, native E4M3 scale atoms
+  kCodecInt4 = 2,    // INT4 codes as E4M3 bytes [M][K], fp32 scales [K/64][ceil(M/128)*128]
+};
+
+// The INT4 recipe (walkthrough eq. (1) with q_max = 7, one fp16 scale per 64
+// elements) for 16 fp32 values a thread holds of a 64-element group; the
+// group's four quarters sit in the four lanes of a quad (lane ^ 1, lane ^ 2):
+//   s = fp16_rne(min(fp32(max|v| / 7), 65504));
+//   q = clamp(rint(fp32(v * fp32(1/s))), -7, 7), all 0 when s is 0.
+// Codes are written as the E4M3 bytes of the integers (exact), the form the
+// FP8 tensor-core MMA reads; the scale is returned as its fp32 value.
+// Every lane of the warp must call it (quad shuffles).
+__device__ __forceinline__ void int4_encode_quarter(const float2 (&v)[8], uint4& codes, float& scale) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fmaxf(fabsf(v[i].x), fabsf(v[i].y)));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 2));
+  const float s = __half2float(__float2half_rn(fminf(__fdiv_rn(amax, 7.0f), 65504.0f)));
+  scale = s;
+  if (s == 0.f) {
+    codes = make_uint4(0u, 0u, 0u, 0u);
+    return;
+  }
+  const float inv = __frcp_rn(s);
+  uint32_t b[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float2 p = mul2_rn(v[i], make_float2(inv, inv));
+    // rint is half-to-even; adding +0 turns a -0 into +0 (code 0 is one byte, 0x00)
+    const float2 qv = make_float2(__fadd_rn(fmaxf(fminf(rintf(p.x), 7.f), -7.f), 0.f),
+                                  __fadd_rn(fmaxf(fminf(rintf(p.y), 7.f), -7.f), 0.f));
+    b[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
+  }
+  codes = make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
+}
+
+// The activation side: v = fp32(x * inv_lambda) for 8 packed bf16 pairs, then
+// int4_encode_quarter.
+__device__ __forceinline__ void encode_int4_quarter(const uint32_t* w, const float* il, uint4& codes, float& scale) {
+  float2 v[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 l = *reinterpret_cast<const float4*>(il + 4 * q);
+    v[2 * q] = mul2_rn(make_float2(bf16lo(w[2 * q]), bf16hi(w[2 * q])), make_float2(l.x, l.y));
+    v[2 * q + 1] = mul2_rn(make_float2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1])), make_float2(l.z, l.w));
+  }
+  int4_encode_quarter(v, codes, scale);
+}
+
+template <int RANK, int BM, int CODEC>
 __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma_kernel(
     const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
     const float* __restrict__ inv_lambda, uint8_t* __restrict__ Qx, uint8_t* __restrict__ Sx,
     __nv_bfloat16* __restrict__ T, int M, int K, int ksplit) {
+  constexpr bool QUANT = CODEC != kCodecNone;
   if constexpr (!QUANT && RANK == 0) return;
   using L = QuantSmem<RANK, BM>;
   constexpr int RG = L::kRowGroups;
@@ -156,7 +212,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
     mbar_init(acc_bar, 1);
     fence_mbar_init();
   }
-  if (QUANT && threadIdx.x < 128) {   // fp32(1/s) for every E4M3 byte with the sign bit clear
+  if (CODEC == kCodecNvfp4 && threadIdx.x < 128) {   // fp32(1/s) for every E4M3 byte with the sign bit clear
     const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)threadIdx.x, __NV_E4M3)));
     rcp_tbl[threadIdx.x] = __frcp_rn(sv);
   }
@@ -240,6 +296,22 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
       }
       const int c = (st0 + j) * L::kCols + 64 * h + 16 * t;   // first column of this thread's group
       const float* il = reinterpret_cast<const float*>(st + kQStageXBytes + L::kL1) + 64 * h + 16 * t;
+      if constexpr (CODEC == kCodecInt4) {
+        uint4 qa, qb;
+        float sA, sB;
+        encode_int4_quarter(xa, il, qa, sA);
+        encode_int4_quarter(xb, il, qb, sB);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);       // the stage's shared memory is no longer read
+        if (okA) *reinterpret_cast<uint4*>(Qx + (size_t)rA * K + c) = qa;
+        if (okB) *reinterpret_cast<uint4*>(Qx + (size_t)rB * K + c) = qb;
+        if (t == 0) {   // rows past M (up to the 128-row padding) get zero scales: TMA zero-fills them
+          float* S = reinterpret_cast<float*>(Sx) + (size_t)(c >> 6) * (size_t)((M + 127) & ~127);
+          S[rA] = sA;
+          S[rB] = sB;
+        }
+        continue;
+      }
       uint2 qa, qb;
       uint32_t sbA, sbB;
       encode_group_bf16(xa, il, rcp_tbl, qa, sbA);

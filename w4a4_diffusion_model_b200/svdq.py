@@ -32,6 +32,8 @@ EXPORTS = [
     "svdq_channel_amax", "svdq_prepare_weights", "svdq_prepare_weights_static", "svdq_quantize_act",
     "svdq_linear", "svdq_linear_quantize_next", "svdq_linear_quantize_next_workspace", "svdq_append_lowrank",
     "svdq_selftest_timeout", "svdq_scales_to_canonical", "svdq_check",
+    "svdq_int4_act_sizes", "svdq_int4_weight_sizes", "svdq_int4_quantize_residual", "svdq_int4_quantize_act",
+    "svdq_int4_linear",
 ]
 
 
@@ -86,6 +88,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_linear_quantize_next.restype = st
     lib.svdq_linear_quantize_next_workspace.argtypes = [Shape, ctypes.c_int32, P(sz)]
     lib.svdq_linear_quantize_next_workspace.restype = st
+    lib.svdq_int4_act_sizes.argtypes, lib.svdq_int4_act_sizes.restype = [Shape, P(sz), P(sz), P(sz)], st
+    lib.svdq_int4_weight_sizes.argtypes, lib.svdq_int4_weight_sizes.restype = [Shape, P(sz), P(sz)], st
+    lib.svdq_int4_quantize_residual.argtypes = [Shape, vp, vp, vp, vp, vp, vp, vp]
+    lib.svdq_int4_quantize_residual.restype = st
+    lib.svdq_int4_quantize_act.argtypes, lib.svdq_int4_quantize_act.restype = [Shape, vp, vp, vp, vp, vp, vp, vp], st
+    lib.svdq_int4_linear.argtypes, lib.svdq_int4_linear.restype = [Shape, vp, vp, vp, vp, vp, vp, vp, vp], st
     _lib = lib
     return lib
 
@@ -252,6 +260,71 @@ def svdq_append_lowrank(W: PreparedWeights, A: torch.Tensor, B: torch.Tensor) ->
     _check(load().svdq_append_lowrank(W.shape.c(), extra, _ptr(W.L1p), _ptr(W.L2t), _ptr(A), _ptr(B), _ptr(L1p),
                                       _ptr(L2t), _stream()))
     return PreparedWeights(LayerShape(0, K, N, r + extra), W.Qr, W.Sr, L1p, L2t, W.lam, W.inv_lam)
+
+
+# ---------------------------------------------------------------- INT4 variant
+
+def svdq_int4_act_sizes(shape: LayerShape) -> tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().svdq_int4_act_sizes(shape.c(), ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def svdq_int4_weight_sizes(shape: LayerShape) -> tuple[int, int]:
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().svdq_int4_weight_sizes(shape.c(), ctypes.byref(a), ctypes.byref(b)))
+    return a.value, b.value
+
+
+@dataclass
+class Int4Weights:
+    shape: LayerShape          # M is unused (0)
+    Qr: torch.Tensor           # uint8 [N][K]: E4M3 bytes of the INT4 codes
+    Sr: torch.Tensor           # fp32 [K/64][N]
+    L2t: torch.Tensor | None   # shared with the NVFP4 preparation
+    L1p: torch.Tensor | None
+    inv_lam: torch.Tensor
+
+
+def svdq_int4_prepare_weights(W_lin: torch.Tensor, P: PreparedWeights) -> Int4Weights:
+    """INT4 encoding of the residual of an NVFP4-prepared layer (same smoothing
+    and low-rank factors)."""
+    N, K = W_lin.shape
+    shape = LayerShape(0, K, N, P.shape.rank)
+    qr, sr = svdq_int4_weight_sizes(shape)
+    Qr = torch.empty(N, K, dtype=torch.uint8, device=W_lin.device)
+    Sr = torch.empty(K // 64, N, dtype=torch.float32, device=W_lin.device)
+    assert Qr.numel() == qr and Sr.numel() * 4 == sr
+    _check(load().svdq_int4_quantize_residual(shape.c(), _ptr(W_lin), _ptr(P.lam), _ptr(P.L1p), _ptr(P.L2t), _ptr(Qr),
+                                              _ptr(Sr), _stream()))
+    return Int4Weights(shape, Qr, Sr, P.L2t, P.L1p, P.inv_lam)
+
+
+def svdq_int4_quantize_act(X: torch.Tensor, inv_lambda: torch.Tensor, L1p: torch.Tensor | None, rank: int,
+                           N: int = 128, out: tuple | None = None):
+    """Returns (Qx [M][K] uint8 E4M3 bytes, Sx fp32 [K/64][ceil(M/128)*128], T [M][rank] bf16 or None)."""
+    M, K = X.shape
+    shape = LayerShape(M, K, N, rank)
+    if out is None:
+        Qx = torch.empty(M, K, dtype=torch.uint8, device=X.device)
+        Sx = torch.empty(K // 64, (M + 127) // 128 * 128, dtype=torch.float32, device=X.device)
+        T = torch.empty(M, rank, dtype=torch.bfloat16, device=X.device) if rank else None
+    else:
+        Qx, Sx, T = out
+    _check(load().svdq_int4_quantize_act(shape.c(), _ptr(X), _ptr(inv_lambda), _ptr(L1p), _ptr(Qx), _ptr(Sx), _ptr(T),
+                                         _stream()))
+    return Qx, Sx, T
+
+
+def svdq_int4_linear(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: Int4Weights,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    M = Qx.shape[0]
+    K, N, rank = W.shape.K, W.shape.N, W.shape.rank
+    shape = LayerShape(M, K, N, rank)
+    Y = out if out is not None else torch.empty(M, N, dtype=torch.bfloat16, device=Qx.device)
+    _check(load().svdq_int4_linear(shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t),
+                                   _ptr(Y), _stream()))
+    return Y
 
 
 def svdq_selftest_timeout() -> None:
