@@ -58,6 +58,8 @@ def parse():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    p.add_argument("--codec", default="nvfp4", choices=["nvfp4", "int4"],
+                   help="int4: the INT4 W4A4 variant (64-element groups, fp16 scales) of the same layer")
     p.add_argument("--no-extras", action="store_true", help="skip the cuBLAS / unfused / rank-0 / e2e / CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--extra-json", default=None, help="append per-leg details to this JSONL file")
@@ -102,6 +104,14 @@ def gemm_flops(w: synth.Workload) -> int:
 
 GEMM_SOURCES = ("svdq_gemm.cuh", "svdq_gemm_pair.cuh", "svdq_gemm_common.cuh", "svdq_ptx.cuh")
 QUANT_SOURCES = ("svdq_quant_tma.cuh", "svdq_quant.cuh", "svdq_ptx.cuh")
+INT4_SOURCES = ("svdq_int4.cuh", "svdq_gemm_common.cuh", "svdq_ptx.cuh")
+
+
+def quantize_bytes_int4(w: synth.Workload) -> int:
+    """Algorithmic HBM bytes of one INT4 quantize launch: read X, inv_lambda,
+    L1p; write one code byte per element, fp32 scales (rows padded to 128), T."""
+    Mp = (w.M + 127) // 128 * 128
+    return 2 * w.M * w.K + 4 * w.K + 2 * w.rank * w.K + w.M * w.K + Mp * (w.K // 64) * 4 + 2 * w.M * w.rank
 
 
 def kernel_source_hash(sources=GEMM_SOURCES) -> str:
@@ -217,7 +227,7 @@ def smi_index(local: int) -> str:
 
 
 # --------------------------------------------------------------------------- CPU oracle leg
-def oracle_sample(w: synth.Workload, X_cpu: torch.Tensor, W_cpu: torch.Tensor, rows=64, cols=512):
+def oracle_sample(w: synth.Workload, X_cpu: torch.Tensor, W_cpu: torch.Tensor, rows=64, cols=512, codec="nvfp4"):
     """Set up the oracle's per-call path on a bounded sample: `rows` token rows
     and `cols` output channels of the layer, full K. Returns (fn, flops)."""
     import oracle as O  # only the CPU-baseline / reference legs use the oracle
@@ -233,16 +243,25 @@ def oracle_sample(w: synth.Workload, X_cpu: torch.Tensor, W_cpu: torch.Tensor, r
     U, S, Vt = np.linalg.svd(What_c, full_matrices=False)
     L1p = O.bf16(U[:, :w.rank] * S[:w.rank] / lam32.astype(np.float64)[:, None])
     L2 = O.bf16(Vt[:w.rank])
-    _, qr, sr = O.residual_quantize(Wn[c_idx], lam32, L1p, L2)
+    R32, qr, sr = O.residual_quantize(Wn[c_idx], lam32, L1p, L2)
     Xs = Xn[r_idx]
 
     def fn():
         qx, sx, T = O.quantize_act(Xs, inv32, L1p)
         return O.linear(qx, sx, T, qr, sr, L2)
 
+    if codec == "int4":
+        qr4, sr4 = O.quantize_int4(R32.T)
+        deq_r = O.dequantize_int4(qr4, sr4)
+
+        def fn():  # noqa: F811
+            xhat = Xs.astype(np.float32) * inv32.astype(np.float32)[None, :]
+            qx4, sx4 = O.quantize_int4(xhat)
+            return O.dequantize_int4(qx4, sx4) @ deq_r.T + (Xs @ L1p) @ L2
+
     m, n = len(r_idx), len(c_idx)
     flops = 2 * m * n * w.K + 2 * m * w.rank * (w.K + n)
-    sample = (f"oracle per-call path (quantize + down-projection + dequantized fp64 GEMM + up-projection) "
+    sample = (f"oracle per-call path ({codec} quantize + down-projection + dequantized fp64 GEMM + up-projection) "
               f"on {m} token rows x {n} output channels x K={w.K} of {w.name}; prepare excluded")
     return fn, flops, sample
 
@@ -308,7 +327,7 @@ def run_reference(args):
         return 0
     w = synth.WORKLOADS[args.workload]
     X, W = synth.generate(w)
-    fn, flops, sample = oracle_sample(w, X, W)
+    fn, flops, sample = oracle_sample(w, X, W, codec=args.codec)
     for _ in range(args.warmup):
         fn()
     times = []
@@ -332,6 +351,36 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU leg
+def int4_extras(args, w, step4, X, Y, X_cpu, W_cpu, flops_step, world, rank_id, timed):
+    """e2e and CPU baseline of the INT4 variant: each step uploads its X from
+    pinned host memory into the first input set's buffer, runs the layer and
+    downloads Y (one step at a time)."""
+    n_x = max(5, args.steps // 2)
+    stream = torch.cuda.current_stream()
+    X_host = X_cpu.pin_memory()
+    Y_host = torch.empty(w.M, w.N, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step(i, ev):
+        ev[0].record(stream)
+        X.copy_(X_host, non_blocking=True)
+        step4(0)
+        Y_host.copy_(Y, non_blocking=True)
+        ev[1].record(stream)
+        ev[2].record(stream)
+    ke, _ = timed(n_x, e2e_step)
+    e2e_ms = aggregate_max(sum(ke), world) / n_x
+    e2e = {"value": round(flops_step * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+           "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
+           "ms_per_step": round(e2e_ms, 4), "pipeline": "one step at a time"}
+    cpu = None
+    if rank_id == 0 and world == 1:
+        fn, fl, sample = oracle_sample(w, X_cpu, W_cpu, codec="int4")
+        v, n, el = time_cpu(fn, fl, args.cpu_seconds)
+        cpu = {"value": round(v, 6), "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+               "sample": sample, "repeats": n, "seconds": round(el, 2)}
+    return e2e, cpu
+
+
 def aggregate_max(value: float, world: int) -> float:
     """Max of a per-rank scalar over all ranks (identity at world size 1)."""
     if world <= 1:
@@ -378,9 +427,14 @@ def run_ours(args):
     torch.cuda.synchronize()
     prepare_ms = e_prep[0].elapsed_time(e_prep[1])
 
+    int4 = args.codec == "int4"
     qx_b, sx_b, t_b = S.svdq_act_sizes(S.LayerShape(w.M, w.K, w.N, w.rank))
-    Qx = torch.empty(w.M, w.K // 2, dtype=torch.uint8, device=dev)
-    Sx = torch.empty(sx_b, dtype=torch.uint8, device=dev)
+    if int4:
+        Qx = torch.empty(w.M, w.K, dtype=torch.uint8, device=dev)
+        Sx = torch.empty(w.K // 64, (w.M + 127) // 128 * 128, dtype=torch.float32, device=dev)
+    else:
+        Qx = torch.empty(w.M, w.K // 2, dtype=torch.uint8, device=dev)
+        Sx = torch.empty(sx_b, dtype=torch.uint8, device=dev)
     T = torch.empty(w.M, w.rank, dtype=torch.bfloat16, device=dev) if w.rank else None
     Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream()
@@ -391,8 +445,23 @@ def run_ours(args):
     n_sets = max(2, min(16, -(-2 * L2_BYTES // set_bytes)))
     sets = [(X, P, P0)] + [(X.clone(), clone_weights(P), clone_weights(P0)) for _ in range(n_sets - 1)]
     l2_note = f"rotating {n_sets} input sets (X + prepared weights, {set_bytes / 1e6:.1f} MB each) > 2x L2"
+    # INT4 residual codes of every set (same smoothing and low-rank factors)
+    sets4 = [S.svdq_int4_prepare_weights(W, P_) for _, P_, _ in sets] if int4 else None
+
+    def step4(i=0, ev=None, out=None):
+        X_, P_, _ = sets[i % n_sets]
+        if ev is not None:
+            ev[0].record(stream)
+        S.svdq_int4_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, out=(Qx, Sx, T))
+        if ev is not None:
+            ev[1].record(stream)
+        S.svdq_int4_linear(Qx, Sx, T, sets4[i % n_sets], out=Y if out is None else out)
+        if ev is not None:
+            ev[2].record(stream)
 
     def step(i=0, rank0=False, variant=S.SVDQ_FUSED, ev=None):
+        if int4:
+            return step4(i, ev)
         X_, P_, P0_ = sets[i % n_sets]
         if rank0:
             P_ = P0_
@@ -481,6 +550,12 @@ def run_ours(args):
     k1_ms = statistics.mean(k1)
     achieved = gemm_flops(w) / (k2_ms * 1e-3) / 1e12
     traffic = profiled_traffic(f"svdq_gemm_{w.name}.md", GEMM_SOURCES)
+    sm_hz = ((clocks or {}).get("sm_mhz") or 1900) * 1e6
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    # INT4 GEMM bound: the rescale's two fp32 operations per output element and
+    # 64-group (128 GEMM flops each), 128 fp32 lanes per SM at the sampled clock
+    alu_peak = 64 * 128 * n_sm * sm_hz / 1e12
+    fp8_peak = 2 * peaks["bf16_tflops_sustained"]
     roofline = {"bound": "tensor", "kernel": gemm_kernel_name(w), "achieved": round(achieved, 2),
                 "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                 "traffic": traffic,
@@ -488,16 +563,27 @@ def run_ours(args):
                              f"{peaks['bf16_tflops_sustained']:.1f} TFLOP/s; "
                              f"vs 9000 TFLOP/s datasheet: {achieved / 9000:.4f}; "
                              f"vs {FP4_PER_BF16:g} x burst bf16: {achieved / (FP4_PER_BF16 * peaks['bf16_tflops']):.4f}"}
-    q_gbs = quantize_bytes(w) / (k1_ms * 1e-3) / 1e9
+    if int4:
+        roofline = {"bound": "alu", "kernel": "svdq_int4_gemm_kernel", "achieved": round(achieved, 2),
+                    "peak": round(alu_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / alu_peak, 4),
+                    "traffic": profiled_traffic(f"svdq_int4_gemm_{w.name}.md", INT4_SOURCES),
+                    "peak_note": f"fp32 rescale bound: 2 fp32 operations per output element and 64-group, "
+                                 f"128 fp32 lanes x {n_sm} SMs x {sm_hz / 1e6:.0f} MHz (sampled); "
+                                 f"vs FP8 tensor peak (2 x {peak_src} sustained bf16) {fp8_peak:.0f} TFLOP/s: "
+                                 f"{achieved / fp8_peak:.4f}"}
+    qbytes = quantize_bytes_int4(w) if int4 else quantize_bytes(w)
+    q_gbs = qbytes / (k1_ms * 1e-3) / 1e9
     roofline_q = {"bound": "hbm", "kernel": "quantize_tma_kernel", "achieved": round(q_gbs, 1),
                   "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(q_gbs / peaks["hbm_gbs"], 4),
-                  "traffic": profiled_traffic(f"quantize_tma_{w.name}.md", QUANT_SOURCES),
-                  "algorithmic_bytes": quantize_bytes(w)}
+                  "traffic": None if int4 else profiled_traffic(f"quantize_tma_{w.name}.md", QUANT_SOURCES),
+                  "algorithmic_bytes": qbytes}
 
     extras = {}
     e2e = None
     cpu = None
-    if not args.no_extras:
+    if not args.no_extras and int4:
+        e2e, cpu = int4_extras(args, w, step4, X, Y, X_cpu, W_cpu, flops_step, world, rank_id, timed)
+    elif not args.no_extras:
         n_x = max(5, args.steps // 2)
         # fused, unfused (same arithmetic, separate passes) and no branch (rank 0)
         # interleaved step by step, so that the comparison sees the same clocks
@@ -574,11 +660,6 @@ def run_ours(args):
         int4_gemm_block = timed_block(n_x, lambda i: S.svdq_int4_linear(Qx4, Sx4, T, sets4[i % n_sets], out=Y)) / n_x
         S.svdq_check()
         g4 = statistics.mean(k2i)
-        sm_hz = ((clocks or {}).get("sm_mhz") or 1900) * 1e6
-        # the rescale bound: two fp32 operations per output element and 64-group
-        # (128 GEMM flops), 128 fp32 lanes per SM
-        alu_peak = 64 * 128 * torch.cuda.get_device_properties(dev).multi_processor_count * sm_hz / 1e12
-        fp8_peak = 2 * peaks["bf16_tflops_sustained"]
         extras["int4"] = {
             "layer_ms": round(int4_layer, 4),
             "layer_tflops": round(flops_step / (int4_layer * 1e-3) / 1e12, 1),
@@ -672,9 +753,10 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4+bf16",
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "int4(e4m3 bytes)+bf16" if int4 else "nvfp4+bf16",
             "data": "synthetic",
-            "config": {"workload": w.name, "M_per_gpu": w.M, "K": w.K, "N": w.N, "rank": w.rank, "alpha": w.alpha,
+            "config": {"workload": w.name, "codec": args.codec, "M_per_gpu": w.M, "K": w.K, "N": w.N, "rank": w.rank, "alpha": w.alpha,
                        "global_tokens": w.M * world, "parallelism": f"token-parallel x{world} (weights replicated)",
                        "l2": l2_note},
             "roofline": roofline, "roofline_quantize": roofline_q,

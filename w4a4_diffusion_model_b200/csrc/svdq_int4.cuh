@@ -9,13 +9,13 @@
 //     them exactly, and each 64-element group's integer products run as
 //     tcgen05 kind::f8f6f4 MMAs (two of K = 32) into an fp32 TMEM buffer; the
 //     sums are integers of magnitude <= 64 * 49, so they are exact;
-//   * eight rescale warps read each group's partial tile back and add it to
+//   * twelve rescale warps read each group's partial tile back and add it to
 //     fp32 accumulators in registers with the group's scale pair:
 //     acc += P * fp32(sx * sw) (the product of two fp16 values is exact in
 //     fp32, so each group's term is rounded once, by the fused multiply-add);
 //   * the low-rank up-projection T L2t^T runs as bf16 MMAs (kind::f16) into
 //     one more partial buffer, added with weight 1.
-// Two 256-column partial buffers alternate, so the MMAs of the next group run
+// Two partial buffers alternate, so the MMAs of the next group run
 // while the rescale warps drain the previous one. The rescale arithmetic
 // (two fp32 operations per element and group) bounds the kernel, not the MMAs.
 //
@@ -78,12 +78,35 @@ __device__ __forceinline__ float2 add2_rn(float2 a, float2 b) {
   return d;
 }
 
-// 32 lanes x 8 consecutive fp32 columns -> 8 registers per thread.
-__device__ __forceinline__ void tmem_ld_32x32b_x8(uint32_t taddr, uint32_t (&r)[8]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr)
-               : "memory");
+// 16 lanes x 256 bits, repeated 8 times along the columns: 32 registers per
+// thread, laid out like mma.sync accumulators. For repetition j, thread t holds
+//   r[4j], r[4j+1]:   lane base + t/4,     columns 8j + 2(t%4) + {0, 1}
+//   r[4j+2], r[4j+3]: lane base + t/4 + 8, the same columns.
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// tcgen05.wait::ld that the compiler sees as producing the loaded registers,
+// so that no use of them is scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait_dep(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+        "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+        "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+        "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
 }
 
 // ---------------------------------------------------------------- weights
@@ -115,23 +138,26 @@ __global__ void residual_quantize_int4_kernel(const __nv_bfloat16* __restrict__ 
 }
 
 // ---------------------------------------------------------------- GEMM
+// Tiles of 128 x 192: twelve rescale warps of 64 columns (three per SM
+// sub-partition) hide each other's TMEM-load latency within 128 registers.
 constexpr int kI4BM = 128;
-constexpr int kI4BN = 256;
+constexpr int kI4BN = 192;
 constexpr int kI4KTile = 128;                        // K elements (= bytes) per k-tile: two groups
 constexpr int kI4StageA = kI4BM * 128;               // 16 KB (also T: 128 x 64 bf16)
-constexpr int kI4StageB = kI4BN * 128;               // 32 KB (also L2t: 256 x 64 bf16)
+constexpr int kI4StageB = kI4BN * 128;               // 24 KB (also L2t: 192 x 64 bf16)
 constexpr int kI4StageSx = 2 * kI4BM * 4;            // fp32 [2 groups][128 rows]
-constexpr int kI4StageSw = 2 * kI4BN * 4;            // fp32 [2 groups][256 columns]
-constexpr int kI4StageBytes = kI4StageA + kI4StageB + kI4StageSx + kI4StageSw;   // 51 KB
-constexpr int kI4Stages = 4;
-constexpr int kI4RescaleWarps = 8;                   // warp w: lanes 32 (w % 4).., columns 128 (w / 4)..
-constexpr int kI4Cols = kI4BN / (kI4RescaleWarps / 4);   // 128 accumulator columns per thread
-constexpr int kI4ProducerWarp = 8;
-constexpr int kI4MmaWarp = 9;
-// 10 warps: at most 3 per SM sub-partition (16K registers each), so up to 168
-// registers per thread -- room for 128 fp32 accumulators
-constexpr int kI4Threads = 32 * 10;
-constexpr uint32_t kI4TmemCols = 512;                // two 256-column partial buffers
+constexpr int kI4StageSw = 2 * kI4BN * 4;            // fp32 [2 groups][192 columns]
+constexpr int kI4StageBytes = (kI4StageA + kI4StageB + kI4StageSx + kI4StageSw + 1023) / 1024 * 1024;   // 43 KB
+constexpr int kI4Stages = 5;
+constexpr int kI4RescaleWarps = 12;                  // warp w: lanes 32 (w % 4).., columns 64 (w / 4)..
+constexpr int kI4Cols = kI4BN / (kI4RescaleWarps / 4);   // 64 accumulator columns per thread
+constexpr int kI4ProducerWarp = 12;
+constexpr int kI4MmaWarp = 13;
+// 14 warps: at most 4 per SM sub-partition (16K registers each), so up to 128
+// registers per thread
+constexpr int kI4Threads = 32 * 14;
+constexpr uint32_t kI4TmpStride = 256;               // TMEM columns between the two partial buffers
+constexpr uint32_t kI4TmemCols = 512;
 constexpr int kI4BarOffset = kI4Stages * kI4StageBytes;
 constexpr int kI4SmemBytes = kI4BarOffset + 256 + 1024;   // barriers + alignment slack
 
@@ -201,8 +227,7 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
       bool ok = true;
       for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const int m0 = (tile / tiles_n) * kI4BM, n0 = (tile % tiles_n) * kI4BN;
-        const bool half = n0 + kI4BN > N;     // only 128 weight rows exist
-        const uint32_t sw_bytes = half ? kI4BN * 2u : kI4BN * 4u;
+        const uint32_t sw_bytes = 4u * (uint32_t)min(kI4BN, N - n0);   // the last tile may be partial
         for (int kt = 0; kt < n_kt + n_lr; ++kt, ++it) {
           const int s = it % kI4Stages;
           if (!mbar_wait(empty + s, ((it / kI4Stages) & 1u) ^ 1u, kDevErrTimeoutEmpty)) {
@@ -267,7 +292,7 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
             for (int j = 0; j < 2; ++j) {   // 32 bytes (= 32 E4M3 elements) of K per MMA
               const uint64_t ad = smem_desc(sa + 64 * gi + 32 * j, 16, 1024, kSwizzle128B);
               const uint64_t bd = smem_desc(sb + 64 * gi + 32 * j, 16, 1024, kSwizzle128B);
-              mma_f8(tmem + b * kI4BN, ad, bd, idesc, (uint32_t)j);
+              mma_f8(tmem + b * kI4TmpStride, ad, bd, idesc, (uint32_t)j);
             }
             tc_commit(tfull + b);
           }
@@ -293,7 +318,7 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
           for (int j = 0; j < k16; ++j) {
             const uint64_t ad = smem_desc(sa + 32 * j, 16, 1024, kSwizzle128B);
             const uint64_t bd = smem_desc(sb + 32 * j, 16, 1024, kSwizzle128B);
-            mma_bf16(tmem + b * kI4BN, ad, bd, idesc_lr, (c | j) != 0 ? 1u : 0u);
+            mma_bf16(tmem + b * kI4TmpStride, ad, bd, idesc_lr, (c | j) != 0 ? 1u : 0u);
           }
           tc_commit(empty + s);
         }
@@ -309,11 +334,19 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
     }
   } else {
     // ------------------------------------------------------------------ rescale warps
+    // Warp w reads lane quarter q = w % 4 (rows 32q..32q+31 of the tile) and
+    // column block cb = w / 4 (64 columns) with the 16x256b shape: thread t
+    // owns rows 32q + 16h + t/4 + {0, 8} (h = 0, 1) and columns
+    // 64cb + 8j + 2(t%4) + {0, 1} (j = 0..7), so it needs 16 weight scales and
+    // 4 activation scales per group.
     const int q = warp & 3, cb = warp >> 2;
-    const uint32_t lane_base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kI4Cols * cb);
-    float2 acc[kI4Cols / 2];
+    const int tr = lane >> 2, tc = 2 * (lane & 3);
+    const uint32_t quarter = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(kI4Cols * cb);
+    float2 acc[2][8][2];   // [h][j][row +0 / +8]: a pair of adjacent columns
 #pragma unroll
-    for (int i = 0; i < kI4Cols / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[h][j][0] = acc[h][j][1] = make_float2(0.f, 0.f);
     uint32_t it = 0, u = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
@@ -336,28 +369,28 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
             break;
           }
           tc_fence_after();
-          const float sxm = ssx[gi * kI4BM + 32 * q + lane];
-          const float* swp = ssw + gi * kI4BN + kI4Cols * cb;
+          const float* swp = ssw + gi * kI4BN + kI4Cols * cb + tc;
+          const float* sxp = ssx + gi * kI4BM + 32 * q + tr;
 #pragma unroll
-          for (int c = 0; c < kI4Cols / 8; ++c) {
-            uint32_t v[8];
-            tmem_ld_32x32b_x8(lane_base + b * kI4BN + 8u * c, v);
-            tmem_ld_wait();
-            if (c == kI4Cols / 8 - 1) {   // the partial buffer is read: the next unit's MMAs may overwrite it
+          for (int h = 0; h < 2; ++h) {
+            uint32_t v[32];
+            tmem_ld_16x256b_x8(quarter + ((uint32_t)(16 * h) << 16) + b * kI4TmpStride, v);
+            tmem_ld_wait_dep(v);
+            if (h == 1) {   // the partial buffer is read: the next unit's MMAs may overwrite it
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(tempty + b);
             }
+            const float sx0 = sxp[16 * h], sx8 = sxp[16 * h + 8];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-              const float4 w4 = *reinterpret_cast<const float4*>(swp + 8 * c + 4 * i);
-              const float2 c0 = mul2_rn(make_float2(w4.x, w4.y), make_float2(sxm, sxm));
-              const float2 c1 = mul2_rn(make_float2(w4.z, w4.w), make_float2(sxm, sxm));
-              acc[4 * c + 2 * i] = fma2_rn(make_float2(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1])), c0,
-                                           acc[4 * c + 2 * i]);
-              acc[4 * c + 2 * i + 1] = fma2_rn(
-                  make_float2(__uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3])), c1,
-                  acc[4 * c + 2 * i + 1]);
+            for (int j = 0; j < 8; ++j) {
+              const float2 w2 = *reinterpret_cast<const float2*>(swp + 8 * j);
+              const float2 c0 = mul2_rn(w2, make_float2(sx0, sx0));
+              const float2 c8 = mul2_rn(w2, make_float2(sx8, sx8));
+              acc[h][j][0] = fma2_rn(make_float2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])), c0,
+                                     acc[h][j][0]);
+              acc[h][j][1] = fma2_rn(make_float2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])),
+                                     c8, acc[h][j][1]);
             }
           }
         }
@@ -374,13 +407,16 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < kI4Cols / 16; ++c) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(lane_base + b * kI4BN + 16u * c, v);
-          tmem_ld_wait();
+        for (int h = 0; h < 2; ++h) {
+          uint32_t v[32];
+          tmem_ld_16x256b_x8(quarter + ((uint32_t)(16 * h) << 16) + b * kI4TmpStride, v);
+          tmem_ld_wait_dep(v);
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            acc[8 * c + i] = add2_rn(acc[8 * c + i], make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])));
+          for (int j = 0; j < 8; ++j) {
+            acc[h][j][0] = add2_rn(acc[h][j][0], make_float2(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1])));
+            acc[h][j][1] =
+                add2_rn(acc[h][j][1], make_float2(__uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3])));
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -391,23 +427,25 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
         it += n_lr;
         ++u;
       }
-      // Y row 32q + lane, columns kI4Cols cb .. of the tile
-      const int row = m0 + 32 * q + lane, col0 = n0 + kI4Cols * cb;
-      if (row < M && col0 < N) {
-        uint4* dst = reinterpret_cast<uint4*>(Y + (size_t)row * N + col0);
+      // Y: each (h, j, +0/+8) pair of adjacent columns is one 4-byte store
+      const int col = n0 + kI4Cols * cb + tc;
+      if (n0 + kI4Cols * cb < N) {
 #pragma unroll
-        for (int i = 0; i < kI4Cols / 8; ++i) {
-          uint32_t p[4];
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(acc[4 * i + j].x, acc[4 * i + j].y);
-            p[j] = *reinterpret_cast<const uint32_t*>(&h);
+          for (int r = 0; r < 2; ++r) {
+            const int row = m0 + 32 * q + 16 * h + tr + 8 * r;
+            if (row >= M) continue;
+            __nv_bfloat16* dst = Y + (size_t)row * N + col;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              *reinterpret_cast<__nv_bfloat162*>(dst + 8 * j) = __floats2bfloat162_rn(acc[h][j][r].x, acc[h][j][r].y);
           }
-          dst[i] = make_uint4(p[0], p[1], p[2], p[3]);
-        }
       }
 #pragma unroll
-      for (int i = 0; i < kI4Cols / 2; ++i) acc[i] = make_float2(0.f, 0.f);
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[h][j][0] = acc[h][j][1] = make_float2(0.f, 0.f);
     }
   }
 
