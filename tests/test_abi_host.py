@@ -144,3 +144,31 @@ def test_linear_quantize_next_argument_checks(lib):
     if not torch.cuda.is_available():
         assert lib.svdq_linear_quantize_next(sh, *args, 32, *nxt, good, 1 << 20, None) == 5
         assert lib.svdq_linear_quantize_next_workspace(sh, 32, ctypes.byref(ws)) == 5
+
+
+def test_int4_sizes_and_argument_checks(lib):
+    """The INT4 entry points: byte sizes of the one-byte codes and the
+    group-major fp32 scales, and argument errors reported before any device
+    work."""
+    qx, sx, t = S.svdq_int4_act_sizes(S.LayerShape(4608, 3072, 9216, 32))
+    assert qx == 4608 * 3072 and sx == 48 * 4608 * 4 and t == 4608 * 32 * 2
+    qx, sx, t = S.svdq_int4_act_sizes(S.LayerShape(130, 384, 128, 0))
+    assert qx == 130 * 384 and sx == 6 * 256 * 4 and t == 0          # rows padded to 128
+    qr, sr = S.svdq_int4_weight_sizes(S.LayerShape(0, 12288, 3072, 32))
+    assert qr == 3072 * 12288 and sr == 192 * 3072 * 4
+    good = ctypes.c_void_p(1 << 20)
+    bad = ctypes.c_void_p((1 << 20) + 8)
+    sh = S.Shape(128, 256, 128, 16)
+    assert lib.svdq_int4_quantize_act(S.Shape(128, 200, 128, 16), good, good, good, good, good, good, None) == 2
+    assert lib.svdq_int4_quantize_act(sh, good, good, good, good, good, None, None) == 1      # T missing
+    assert lib.svdq_int4_quantize_act(sh, good, good, good, bad, good, good, None) == 3
+    assert lib.svdq_int4_linear(sh, good, good, good, good, good, None, good, None) == 1      # L2t missing
+    assert lib.svdq_int4_linear(sh, good, good, good, good, bad, good, good, None) == 3
+    assert lib.svdq_int4_linear(S.Shape(128, 256, 100, 0), good, good, None, good, good, None, good, None) == 2
+    assert lib.svdq_int4_quantize_residual(sh, good, good, None, good, good, good, None) == 1  # L1p missing
+    assert lib.svdq_int4_quantize_residual(sh, good, good, good, good, good, bad, None) == 3
+    assert lib.svdq_int4_quantize_act(S.Shape(0, 256, 128, 0), None, None, None, None, None, None, None) == 0
+    if not torch.cuda.is_available():
+        sh0 = S.Shape(128, 256, 128, 0)
+        assert lib.svdq_int4_linear(sh0, good, good, None, good, good, None, good, None) == 5
+        assert lib.svdq_int4_quantize_residual(sh0, good, good, None, None, good, good, None) == 5
