@@ -429,9 +429,13 @@ def run_ours(args):
 
     int4 = args.codec == "int4"
     qx_b, sx_b, t_b = S.svdq_act_sizes(S.LayerShape(w.M, w.K, w.N, w.rank))
+
+    def int4_act_buffers():
+        """INT4 activation codes (one byte each) and group-major fp32 scales."""
+        return (torch.empty(w.M, w.K, dtype=torch.uint8, device=dev),
+                torch.empty(w.K // 64, (w.M + 127) // 128 * 128, dtype=torch.float32, device=dev))
     if int4:
-        Qx = torch.empty(w.M, w.K, dtype=torch.uint8, device=dev)
-        Sx = torch.empty(w.K // 64, (w.M + 127) // 128 * 128, dtype=torch.float32, device=dev)
+        Qx, Sx = int4_act_buffers()
     else:
         Qx = torch.empty(w.M, w.K // 2, dtype=torch.uint8, device=dev)
         Sx = torch.empty(sx_b, dtype=torch.uint8, device=dev)
@@ -445,19 +449,24 @@ def run_ours(args):
     n_sets = max(2, min(16, -(-2 * L2_BYTES // set_bytes)))
     sets = [(X, P, P0)] + [(X.clone(), clone_weights(P), clone_weights(P0)) for _ in range(n_sets - 1)]
     l2_note = f"rotating {n_sets} input sets (X + prepared weights, {set_bytes / 1e6:.1f} MB each) > 2x L2"
-    # INT4 residual codes of every set (same smoothing and low-rank factors)
-    sets4 = [S.svdq_int4_prepare_weights(W, P_) for _, P_, _ in sets] if int4 else None
 
-    def step4(i=0, ev=None, out=None):
-        X_, P_, _ = sets[i % n_sets]
-        if ev is not None:
-            ev[0].record(stream)
-        S.svdq_int4_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, out=(Qx, Sx, T))
-        if ev is not None:
-            ev[1].record(stream)
-        S.svdq_int4_linear(Qx, Sx, T, sets4[i % n_sets], out=Y if out is None else out)
-        if ev is not None:
-            ev[2].record(stream)
+    def make_step4(Qx_, Sx_):
+        """One INT4 layer step on input set i (INT4 residual codes of every set,
+        same smoothing and low-rank factors); events as in step()."""
+        sets4 = [S.svdq_int4_prepare_weights(W, P_) for _, P_, _ in sets]
+
+        def step4(i=0, ev=None):
+            X_, P_, _ = sets[i % n_sets]
+            if ev is not None:
+                ev[0].record(stream)
+            S.svdq_int4_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, out=(Qx_, Sx_, T))
+            if ev is not None:
+                ev[1].record(stream)
+            S.svdq_int4_linear(Qx_, Sx_, T, sets4[i % n_sets], out=Y)
+            if ev is not None:
+                ev[2].record(stream)
+        return step4, sets4
+    step4 = make_step4(Qx, Sx)[0] if int4 else None
 
     def step(i=0, rank0=False, variant=S.SVDQ_FUSED, ev=None):
         if int4:
@@ -637,26 +646,13 @@ def run_ours(args):
         extras["lowrank_overhead_gemm"] = round(statistics.mean(k2f) / extras["rank0_gemm_ms"] - 1, 4)
         extras["unfused_overhead_layer"] = round(extras["unfused_layer_ms"] / extras["rank0_layer_ms"] - 1, 4)
 
-        # the INT4 variant (64-element groups, fp16 scales) of the same layer:
-        # same smoothing and low-rank factors, INT4 residual and activation
-        sets4 = [S.svdq_int4_prepare_weights(W, P_) for _, P_, _ in sets]
-        Qx4 = torch.empty(w.M, w.K, dtype=torch.uint8, device=dev)
-        Sx4 = torch.empty(w.K // 64, (w.M + 127) // 128 * 128, dtype=torch.float32, device=dev)
-
-        def step4(i, ev=None):
-            X_, P_, _ = sets[i % n_sets]
-            if ev is not None:
-                ev[0].record(stream)
-            S.svdq_int4_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, out=(Qx4, Sx4, T))
-            if ev is not None:
-                ev[1].record(stream)
-            S.svdq_int4_linear(Qx4, Sx4, T, sets4[i % n_sets], out=Y)
-            if ev is not None:
-                ev[2].record(stream)
+        # the INT4 variant (64-element groups, fp16 scales) of the same layer
+        Qx4, Sx4 = int4_act_buffers()
+        step4c, sets4 = make_step4(Qx4, Sx4)
         for i in range(3):
-            step4(i)
-        int4_layer = timed_block(n_x, lambda i: step4(i)) / n_x
-        k1i, k2i = timed(n_x, lambda i, ev: step4(i, ev), warm=0)
+            step4c(i)
+        int4_layer = timed_block(n_x, lambda i: step4c(i)) / n_x
+        k1i, k2i = timed(n_x, lambda i, ev: step4c(i, ev), warm=0)
         int4_gemm_block = timed_block(n_x, lambda i: S.svdq_int4_linear(Qx4, Sx4, T, sets4[i % n_sets], out=Y)) / n_x
         S.svdq_check()
         g4 = statistics.mean(k2i)

@@ -319,3 +319,39 @@ def test_native_scales_of_quantized_activation_roundtrip():
     L = O.layer_reference(X, W_lin, 0.5, r)
     nat = O.scales_to_native(L["Sx"])
     assert np.array_equal(O.native_to_scales(nat, X.shape[0], X.shape[1]), L["Sx"])
+
+
+def test_eq7_eq8_gaussian_residual_monte_carlo():
+    """Walkthrough eq. (7)/(8) with its Gaussian constant
+    c = sqrt(pi log(size) / size) (Gaussian maximal inequality and the
+    half-normal mean): on iid normal matrices E[max|R|] <= c E[||R||_F], and
+    each of the oracle's 4-bit quantizers keeps
+    E[||R - Q(R)||_F] <= c sqrt(size) / q_max E[||R||_F] (per-tensor INT4,
+    NVFP4 groups of 16 with q_max = 6, INT4 groups of 64 with q_max = 7).
+    The two uniform quantizers also match the uniform-rounding error
+    E||R - Q(R)||^2 = sum over elements of step^2 / 12 within 5 %, which pins
+    their step sizes (max/7 per tensor, the fp16 group scale per 64)."""
+    rng = np.random.default_rng(21)
+    for shape in ((64, 64), (128, 512), (512, 1024)):
+        size = shape[0] * shape[1]
+        c = math.sqrt(math.pi * math.log(size) / size)
+        Rs = [(rng.standard_normal(shape) * 0.37).astype(np.float32).astype(np.float64) for _ in range(12)]
+        m_max = np.mean([np.abs(R).max() for R in Rs])
+        m_fro = np.mean([O.fro(R) for R in Rs])
+        assert m_max <= c * m_fro
+        quantizers = {
+            "int4 per tensor": (7, lambda R: O.fake_quant_int(R, 4)),
+            "nvfp4 g16": (6, lambda R: O.dequantize_nvfp4(*O.quantize_nvfp4(R))),
+            "int4 g64": (7, lambda R: O.dequantize_int4(*O.quantize_int4(R))),
+        }
+        for name, (qmax, q) in quantizers.items():
+            m_err = np.mean([O.fro(R - q(R)) for R in Rs])
+            assert m_err <= c * math.sqrt(size) / qmax * m_fro, name
+        # uniform rounding: error variance step^2 / 12 per element
+        for R in Rs[:4]:
+            err2 = O.fro(R - O.fake_quant_int(R, 4)) ** 2
+            step = np.abs(R).max() / 7
+            assert abs(err2 / (size * step ** 2 / 12) - 1) < 0.05
+            _, s = O.quantize_int4(R)
+            err2 = O.fro(R - O.dequantize_int4(*O.quantize_int4(R))) ** 2
+            assert abs(err2 / (64 * np.sum(s ** 2) / 12) - 1) < 0.05
