@@ -126,3 +126,23 @@ def test_our_arm_fails_loudly_without_a_device():
                          timeout=300, cwd=ROOT)
     assert out.returncode != 0
     assert not any(s.startswith("{") for s in out.stdout.splitlines())
+
+
+def test_reference_arm_int4_codec():
+    """`--codec int4` times the oracle's INT4 per-call path (the same line
+    contract as the NVFP4 reference arm)."""
+    cmd = [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--codec", "int4", "--steps", "2",
+           "--warmup", "1", "--workload", synth.TINY.name]
+    out = subprocess.run(cmd, capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    d = [json.loads(s) for s in out.stdout.splitlines() if s.startswith("{")][-1]
+    assert d["impl"] == "reference" and d["value"] > 0
+    assert "int4" in d["cpu_baseline"]["sample"]
+
+
+def test_int4_quantize_bytes():
+    w = synth.FLUX_QKV
+    # X read, inv_lambda, L1p read; one byte per code, fp32 scales per 64 (rows padded to 128), T written
+    assert bench.quantize_bytes_int4(w) == (2 * 4608 * 3072 + 4 * 3072 + 2 * 32 * 3072 + 4608 * 3072
+                                            + 4608 * 48 * 4 + 2 * 4608 * 32)
+    assert bench.quantize_bytes_int4(w.with_(M=130)) - bench.quantize_bytes_int4(w.with_(M=129)) == 2 * 3072 + 3072 + 64
