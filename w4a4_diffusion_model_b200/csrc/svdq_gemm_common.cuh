@@ -118,7 +118,7 @@ __device__ __forceinline__ void epilogue_store_band(const uint32_t (&p)[32 * BOX
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0 && store) {
-      tma_store_2d(tm_y, box, col0 + 64 * b, row0);
+      tma_store_2d_evict_first(tm_y, box, col0 + 64 * b, row0);   // Y is not read again here
       bulk_commit();
     }
   }

@@ -172,6 +172,17 @@ __device__ __forceinline__ void tma_store_2d(const void* tmap, const void* src, 
                : "memory");
 }
 
+// The same store, its lines marked first for eviction from L2: an output the
+// kernel does not read again is then written back while the kernel runs, not
+// when a later kernel's reads need the space.
+__device__ __forceinline__ void tma_store_2d_evict_first(const void* tmap, const void* src, int x, int y) {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+               ::"l"(tmap), "r"(smem_u32(src)), "r"(x), "r"(y), "l"(pol)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 template <int N>
