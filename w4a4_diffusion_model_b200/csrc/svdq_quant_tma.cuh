@@ -76,6 +76,19 @@ struct QuantSmem {
   static constexpr int kBytes = kBarOffset + 256 + 1024;
 };
 
+// TMA load of a 2-D box whose lines are marked first for eviction from L2:
+// the quantizer reads each element of X exactly once, so X should not push
+// the next kernel's operands out of L2.
+__device__ __forceinline__ void tma_load_2d_once(void* dst, const void* tmap, uint64_t* bar, int x, int y) {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%3, %4}], [%2], %5;"
+      ::"r"(smem_u32(dst)), "l"(tmap), "r"(smem_u32(bar)), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
+
 // Byte offset of 16-byte chunk c of row r in a 128B-swizzled box (128-byte rows).
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
@@ -240,7 +253,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
         mbar_arrive_expect_tx(full + s, (uint32_t)(kQStageXBytes + L::kL1 + (QUANT ? L::kInv : 0)));
 #pragma unroll
         for (int b = 0; b < L::kSlabs; ++b) {
-          tma_load_2d(st + b * L::kBoxBytes, &tm_x, full + s, c0 + 64 * b, m0);
+          tma_load_2d_once(st + b * L::kBoxBytes, &tm_x, full + s, c0 + 64 * b, m0);
           if (RANK > 0) tma_load_2d(st + kQStageXBytes + b * L::kL1Box, &tm_l1, full + s, c0 + 64 * b, 0);
         }
         if (QUANT) bulk_load(st + kQStageXBytes + L::kL1, inv_lambda + c0, (uint32_t)L::kInv, full + s);
