@@ -95,3 +95,23 @@ def test_int4_codes_as_e4m3_bytes_match_torch():
     lib = torch.tensor(ints, dtype=torch.float32).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(ours, lib)
     assert np.array_equal(O.e4m3_decode(ours), ints.astype(np.float64))
+
+
+def test_int4_layer_output_brute_force_tiny():
+    """layer_reference_int4's Y against a plain-Python loop over its own codes,
+    scales and factors: Y[m][n] = sum_k qx sx(m, k/64) qr sr(n, k/64)
+    + sum_j T[m][j] L2[j][n]."""
+    rng = np.random.default_rng(31)
+    M, K, N, r = 3, 128, 4, 2
+    X = O.bf16(rng.standard_normal((M, K)) * np.exp(rng.uniform(-1, 1, K)))
+    W = O.bf16(rng.standard_normal((N, K)) / np.sqrt(K))
+    ref = O.layer_reference_int4(X, W, 0.5, r)
+    qx, sx, qr, sr, T, L2 = ref["Qx4"], ref["Sx4"], ref["Qr4"], ref["Sr4"], ref["T"], ref["L2"]
+    for m in range(M):
+        for n in range(N):
+            acc = 0.0
+            for k in range(K):
+                acc += float(qx[m, k]) * float(sx[m, k // 64]) * float(qr[n, k]) * float(sr[n, k // 64])
+            for j in range(r):
+                acc += float(T[m, j]) * float(L2[j, n])
+            assert abs(acc - ref["Y"][m, n]) <= 1e-12 * max(1.0, abs(acc))
