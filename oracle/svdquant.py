@@ -12,6 +12,8 @@ precision), what the layer computes:
     W_hat = diag(lambda) W = L1 L2 + R
 
 Sources (web pages on SVDQuant):
+  [P1] libaedu.com, article on 4-bit diffusion-model quantization (smoothing,
+       kernel fusion, and the DeltaQuant core + delta outline for video).
   [P2] devpress.csdn.net, SVDQuant paper walkthrough: eq. (1) symmetric
        quantization with q_max = 6 for 4-bit float, eq. (2) the factored W4A4
        product, eq. (3) the error E, eq. (4)/(9) Proposition 4.1, eq. (5) the
@@ -56,6 +58,7 @@ __all__ = [
     "quant_error", "prop41_bound", "rel_fro", "fro",
     "INT4_QMAX", "INT4_GROUP", "fp16", "quantize_int4", "dequantize_int4", "pack_int4", "unpack_int4",
     "layer_reference_int4",
+    "e4m3_encode_signed", "video_blocks", "deltaquant_encode", "deltaquant_decode",
 ]
 
 # ---------------------------------------------------------------------------
@@ -418,6 +421,61 @@ def layer_reference_int4(X, W_lin, alpha: float, rank: int, act_amax=None) -> di
     if rank:
         Y = Y + T @ P["L2"]
     return {**P, "Qx4": Qx, "Sx4": Sx, "Qr4": Qr, "Sr4": Sr, "T": T, "Y": Y, "Y_exact": X @ np.asarray(W_lin, np.float64).T}
+
+
+# ---------------------------------------------------------------------------
+# DeltaQuant-style core + delta activations ([P1] libaedu.com article on
+# 4-bit diffusion-model quantization, DeltaQuant paragraphs: video
+# activations are split into local 3-D spatio-temporal blocks; each block's
+# mean token is the core token, kept in FP8; the differences to it are
+# quantized to 4 bits). The page gives the method in outline only. Readings:
+#   * tokens of a video latent [F][H][Wd] are rows in frame, row, column
+#     order; blocks are bf x bh x bw tokens (default 2 x 2 x 2), tiled from
+#     the origin; blocks at a ragged edge hold the tokens that exist;
+#   * core = E4M3_RNE_satfinite of the block's exact mean (fp64), per channel,
+#     with no scale (the page names FP8 and nothing else);
+#   * delta = fp32(x - decode(core)), i.e. relative to the stored core, so
+#     the core's rounding is absorbed by the delta; deltas are NVFP4 (groups of
+#     16 channels, the codec above);
+#   * reconstruction x~ = decode(core) + deq(delta).
+# Oracle only: no kernel consumes this encoding yet.
+
+def e4m3_encode_signed(v) -> np.ndarray:
+    """E4M3 byte of RNE_satfinite(v) for any sign (sign bit 0x80; a negative
+    value that rounds to zero keeps it)."""
+    v = np.asarray(v, dtype=np.float64)
+    mag = e4m3_encode(np.abs(v)).astype(np.int64)
+    return (mag | np.where(np.signbit(v), 0x80, 0)).astype(np.uint8)
+
+
+def video_blocks(F: int, H: int, Wd: int, block=(2, 2, 2)) -> np.ndarray:
+    """Block index of every token (rows in frame, row, column order)."""
+    bf, bh, bw = block
+    nbh, nbw = -(-H // bh), -(-Wd // bw)
+    f, h, w = np.meshgrid(np.arange(F), np.arange(H), np.arange(Wd), indexing="ij")
+    return ((f // bf) * nbh * nbw + (h // bh) * nbw + (w // bw)).reshape(-1)
+
+
+def deltaquant_encode(X: np.ndarray, dims, block=(2, 2, 2)) -> dict:
+    """Core tokens (E4M3 bytes, [blocks][C]) and NVFP4 deltas of X [F*H*Wd][C]."""
+    X = np.asarray(X, dtype=np.float64)
+    F, H, Wd = dims
+    assert X.shape[0] == F * H * Wd and X.shape[1] % 16 == 0
+    blk = video_blocks(F, H, Wd, block)
+    nb = int(blk.max()) + 1
+    sums = np.zeros((nb, X.shape[1]))
+    np.add.at(sums, blk, X)
+    counts = np.bincount(blk, minlength=nb).astype(np.float64)
+    core_codes = e4m3_encode_signed(sums / counts[:, None])
+    core = e4m3_decode(core_codes)
+    delta = fp32(X - core[blk])
+    codes, scales = quantize_nvfp4(delta)
+    return dict(block_of_token=blk, core_codes=core_codes, delta_codes=codes, delta_scales=scales)
+
+
+def deltaquant_decode(enc: dict) -> np.ndarray:
+    core = e4m3_decode(enc["core_codes"])
+    return core[enc["block_of_token"]] + dequantize_nvfp4(enc["delta_codes"], enc["delta_scales"])
 
 
 def fake_quant_int(x: np.ndarray, bits: int, axis=None) -> np.ndarray:

@@ -19,7 +19,8 @@ Recipe (one numpy PCG64 stream per workload, draws taken in the order below):
   even) by torch's dtype conversion; every consumer sees the bf16 values.
 
 These stand in for FLUX.1 activations and weights (the workloads the SVDQuant
-paper measures), which are not available offline.
+paper measures), which are not available offline. ``smooth_video`` draws a
+spatio-temporally smooth activation for the core + delta video codec.
 """
 from __future__ import annotations
 
@@ -122,3 +123,24 @@ def generate(w: Workload, M: int | None = None) -> tuple[torch.Tensor, torch.Ten
     X = make_activation(w, rng, M)
     W = make_weight(w, rng)
     return X, W
+
+
+def smooth_video(F: int, H: int, Wd: int, C: int, seed: int, noise: float = 0.05,
+                 outlier_channels: int = 2) -> torch.Tensor:
+    """A video-latent-like activation, tokens as rows in frame, row, column
+    order ([F*H*Wd][C] bf16): per channel, a sum of four low-frequency
+    separable cosines over (frame, row, column) with random frequencies below
+    a quarter cycle per token and random phases, plus i.i.d. N(0, noise^2);
+    the first ``outlier_channels`` channels are scaled by 20."""
+    rng = np.random.default_rng(seed)
+    f = np.arange(F)[:, None, None, None]
+    h = np.arange(H)[None, :, None, None]
+    w = np.arange(Wd)[None, None, :, None]
+    x = np.zeros((F, H, Wd, C))
+    for _ in range(4):
+        kf, kh, kw = (rng.uniform(0.0, 0.25, C) * 2 * np.pi for _ in range(3))
+        ph = rng.uniform(0.0, 2 * np.pi, C)
+        x += rng.standard_normal(C) * np.cos(kf * f + kh * h + kw * w + ph)
+    x += noise * rng.standard_normal(x.shape)
+    x[..., :outlier_channels] *= 20.0
+    return _to_bf16(x.reshape(F * H * Wd, C))
