@@ -28,11 +28,15 @@ Sources (web pages on SVDQuant):
 Readings where the pages leave a step open (each one is also listed in the
 design notes of the repository):
   * NVFP4 = one E4M3 scale per 16 consecutive elements along the reduction
-    dimension, scale = E4M3_RNE_satfinite(fp32(amax / 6)); no second-level
+    dimension, scale s = E4M3_RNE_satfinite(amax / 6); no second-level
     per-tensor scale.
-  * codes: q = E2M1_RNE_satfinite(fp32(v * fp32(1 / s))), sign-preserving
-    (a negative value that rounds to zero keeps the sign bit); a group whose
-    scale is zero encodes all +0.
+  * codes: q = E2M1_RNE_satfinite(v / s) of the exact real quotient ([P2]
+    eq. (1), round(X / s)), sign-preserving (a negative value that rounds to
+    zero keeps the sign bit); a group whose scale is zero encodes all +0.
+  * "round to nearest, ties to even" of an exact quotient num / den onto a
+    grid is taken by comparing |num| with each grid midpoint times den; those
+    products are exact in fp64 for every grid and divisor used here, so no
+    intermediate rounding of the quotient enters any decision.
   * smoothing: lambda64 = ax^alpha / aw^(1-alpha) (alpha = 0.5 uses sqrt on
     both sides), lambda = 1 where ax or aw is zero; lambda32 = fp32(lambda64),
     inv_lambda32 = fp32(1 / lambda32).
@@ -54,7 +58,8 @@ __all__ = [
     "scales_to_native", "native_to_scales",
     "channel_amax", "smoothing_lambda", "prepare_weights", "residual_quantize",
     "quantize_act", "linear", "layer_reference",
-    "fake_quant_int", "smooth_fp", "svdquant_fakequant",
+    "int_quant_dequant", "smoothed_pair", "fakequant_output", "lambda64", "svd_split",
+    "rne_quotient_index", "E4M3_GRID", "FP16_GRID", "INT4_GRID",
     "quant_error", "prop41_bound", "rel_fro", "fro",
     "INT4_QMAX", "INT4_GROUP", "fp16", "quantize_int4", "dequantize_int4", "pack_int4", "unpack_int4",
     "layer_reference_int4",
@@ -147,6 +152,9 @@ def e4m3_encode(v) -> np.ndarray:
     return (ebits.astype(np.int64) << 3 | mbits.astype(np.int64)).astype(np.uint8)
 
 
+E4M3_BYTES_FINITE = np.arange(127, dtype=np.uint8)            # 0x00..0x7e: every finite value >= 0
+
+
 # ---------------------------------------------------------------------------
 # NVFP4 group quantization ([P2] eq. (1) with q_max = 6, Table 3's microscaling)
 # ---------------------------------------------------------------------------
@@ -154,27 +162,63 @@ def e4m3_encode(v) -> np.ndarray:
 GROUP = 16
 
 
+def rne_quotient_index(num, den, grid: np.ndarray) -> np.ndarray:
+    """Index into ``grid`` of RNE_satfinite(|num| / den), the quotient taken
+    exactly.
+
+    ``grid`` holds the non-negative values of a format in ascending order, so
+    that an even index is an even code. Midpoint i lies between grid[i] and
+    grid[i + 1]; |num| passes it when |num| > mid_i * den, and on a tie
+    (|num| == mid_i * den) exactly when i + 1 is even. Quotients above the
+    last midpoint take the last grid value (saturation). ``den`` is a positive
+    scalar or an array broadcasting against ``num`` on all but its last axis
+    (one divisor per group of the last axis). Each product mid_i * den must be
+    exact in fp64, which the callers guarantee (few significant bits on both
+    sides).
+    """
+    a = np.abs(np.asarray(num, dtype=np.float64))
+    grid = np.asarray(grid, dtype=np.float64)
+    mids = (grid[:-1] + grid[1:]) / 2                       # exact in fp64
+    if np.ndim(den) == 0:
+        t = mids * float(den)
+        i = np.searchsorted(t, a, side="left")              # midpoints strictly below |num|
+        j = np.minimum(i, t.size - 1)
+        tie_up = (i < t.size) & (t[j] == a) & ((i + 1) % 2 == 0)
+        return (i + tie_up).astype(np.int64)
+    d = np.asarray(den, dtype=np.float64)[..., None]
+    idx = np.zeros(a.shape, dtype=np.int64)
+    for i, mu in enumerate(mids):                           # thresholds ascend with i
+        t = mu * d
+        passed = a > t
+        if (i + 1) % 2 == 0:
+            passed |= a == t
+        idx += passed
+    return idx
+
+
+E4M3_GRID = e4m3_decode(E4M3_BYTES_FINITE)                     # ascending; index = byte
+
+
 def quantize_nvfp4(v32: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
     """Quantize rows of fp32 values, grouped by 16 along the last axis.
 
     Returns (codes uint8 [rows][K] one nibble per element, scales uint8
-    [rows][K/16] E4M3 bytes). Steps, per group: a = max|v|;
-    s = E4M3(fp32(a / 6)); q = E2M1(fp32(v * fp32(1 / s))); all +0 if s == 0.
+    [rows][K/16] E4M3 bytes). Per group ([P2] eq. (1) with q_max = 6):
+    a = max|v|; s = E4M3_RNE_satfinite(a / 6); q = E2M1_RNE_satfinite(v / s),
+    both quotients exact; all codes +0 if s == 0.
     """
-    v = np.asarray(v32, dtype=np.float32)
+    v = np.asarray(v32, dtype=np.float32).astype(np.float64)
     rows, K = v.shape
     if K % GROUP:
         raise ValueError("K must be a multiple of 16")
     g = v.reshape(rows, K // GROUP, GROUP)
     amax = np.max(np.abs(g), axis=2)                                 # exact
-    s32 = amax / np.float32(E2M1_QMAX)                               # IEEE fp32 divide
-    sbyte = e4m3_encode(s32.astype(np.float64))
-    sval = e4m3_decode(sbyte).astype(np.float32)                     # exact in fp32
-    with np.errstate(divide="ignore", invalid="ignore"):
-        inv = np.float32(1.0) / sval                                 # IEEE fp32 reciprocal
-        y = g * inv[..., None]                                       # fp32 multiply
-    codes = e2m1_encode(y.astype(np.float64))
-    codes = np.where((sval == 0)[..., None], np.uint8(0), codes)
+    sbyte = rne_quotient_index(amax, E2M1_QMAX, E4M3_GRID).astype(np.uint8)
+    sval = e4m3_decode(sbyte)
+    live = sval > 0
+    mag = rne_quotient_index(g, np.where(live, sval, 1.0), E2M1_VALUES).astype(np.uint8)
+    codes = mag | (np.signbit(g).astype(np.uint8) << 3)
+    codes = np.where(live[..., None], codes, np.uint8(0))
     return codes.reshape(rows, K).astype(np.uint8), sbyte
 
 
@@ -237,21 +281,28 @@ def channel_amax(X: np.ndarray) -> np.ndarray:
     return np.max(np.abs(np.asarray(X, dtype=np.float64)), axis=0).astype(np.float32)
 
 
+def lambda64(ax, aw, alpha: float) -> np.ndarray:
+    """lambda_j = ax_j^alpha / aw_j^(1-alpha) in fp64 ([P3] SmoothQuant
+    section), 1 where either channel maximum is 0. alpha = 0.5 takes a square
+    root on each side."""
+    ax = np.asarray(ax, dtype=np.float64)
+    aw = np.asarray(aw, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        if alpha == 0.5:
+            lam = np.sqrt(ax) / np.sqrt(aw)
+        else:
+            lam = np.power(ax, alpha) / np.power(aw, 1.0 - alpha)
+    return np.where((ax == 0) | (aw == 0), 1.0, lam)
+
+
 def smoothing_lambda(act_amax: np.ndarray, W_lin: np.ndarray, alpha: float):
     """lambda_j = max|X_j|^alpha / max|W_j|^(1-alpha), W_j = input channel j.
 
     W_lin is [N][K] (nn.Linear); the paper's W = W_lin^T, so channel j of the
     weight is column j of W_lin. Returns (lambda32, inv_lambda32) as float32.
     """
-    ax = np.asarray(act_amax, dtype=np.float64)
     aw = np.max(np.abs(np.asarray(W_lin, dtype=np.float64)), axis=0)
-    with np.errstate(divide="ignore", invalid="ignore"):
-        if alpha == 0.5:
-            lam = np.sqrt(ax) / np.sqrt(aw)
-        else:
-            lam = np.power(ax, alpha) / np.power(aw, 1.0 - alpha)
-    lam = np.where((ax == 0) | (aw == 0), 1.0, lam)
-    lam32 = lam.astype(np.float32)
+    lam32 = lambda64(act_amax, aw, alpha).astype(np.float32)
     inv32 = np.float32(1.0) / lam32
     return lam32, inv32
 
@@ -282,6 +333,14 @@ def residual_quantize(W_lin: np.ndarray, lam32: np.ndarray, L1p: np.ndarray, L2:
     return R32, codes, scales
 
 
+def svd_split(What: np.ndarray, rank: int):
+    """Top-rank split of W_hat [K][N] by the SVD ([P2] text after eq. (8):
+    the optimal rank-r approximation; [P3] SVDQuant section): L1 = U_r
+    diag(S_r) [K][r], L2 = V_r^T [r][N], and all singular values (descending)."""
+    U, S, Vt = np.linalg.svd(What, full_matrices=False)
+    return U[:, :rank] * S[:rank], Vt[:rank], S
+
+
 def prepare_weights(W_lin: np.ndarray, act_amax: np.ndarray, alpha: float, rank: int) -> dict:
     """Offline preparation: smoothing, top-r SVD split, residual quantization.
 
@@ -292,10 +351,9 @@ def prepare_weights(W_lin: np.ndarray, act_amax: np.ndarray, alpha: float, rank:
     W = np.asarray(W_lin, dtype=np.float64)
     lam32, inv32 = smoothing_lambda(act_amax, W, alpha)
     What = lam32.astype(np.float64)[:, None] * W.T
-    U, S, Vt = np.linalg.svd(What, full_matrices=False)
-    L1 = U[:, :rank] * S[:rank]
+    L1, L2_64, S = svd_split(What, rank)
     L1p = bf16(L1 / lam32.astype(np.float64)[:, None])
-    L2 = bf16(Vt[:rank])
+    L2 = bf16(L2_64)
     R32, codes, scales = residual_quantize(W, lam32, L1p, L2)
     return dict(lam32=lam32, inv32=inv32, L1p=L1p, L2=L2, S=S, R32=R32,
                 Qr=codes, Sr=scales, What=What)
@@ -348,12 +406,14 @@ def layer_reference(X, W_lin, alpha: float, rank: int, act_amax=None) -> dict:
 # ---------------------------------------------------------------------------
 # INT4 W4A4 variant (the pages' path for GPUs without NVFP4: [P2] eq. (1) with
 # q_max = 2^(k-1) - 1 = 7 for signed 4-bit integers; [P3] "one scale per 64
-# elements"). Readings: fp16 scales, s = fp16_RNE(fp32(amax / 7)) saturating at
-# 65504; q = clamp(RNE(fp32(v * fp32(1/s))), -7, 7) (the same multiply-by-the-
-# rounded-reciprocal recipe as the NVFP4 codes); a zero scale gives zero codes.
+# elements"). Readings: fp16 scales, s = fp16_RNE(amax / 7) saturating at
+# 65504; q = clamp(RNE(v / s), -7, 7), both quotients exact (eq. (1)'s
+# round(X / s)); a zero scale gives zero codes.
 
 INT4_QMAX = 7
 INT4_GROUP = 64
+FP16_GRID = np.arange(0x7C00, dtype=np.uint16).view(np.float16).astype(np.float64)   # 0 .. 65504, index = bits
+INT4_GRID = np.arange(INT4_QMAX + 1, dtype=np.float64)                                  # 0 .. 7
 
 
 def fp16(v) -> np.ndarray:
@@ -365,18 +425,16 @@ def quantize_int4(v32: np.ndarray, group: int = INT4_GROUP) -> tuple[np.ndarray,
     """Symmetric INT4 group quantization along the last axis of fp32 values.
 
     Returns (codes int8 in [-7, 7], scales as fp16 values in float64 [.., K/group])."""
-    v = np.asarray(v32, dtype=np.float64)
+    v = np.asarray(v32, dtype=np.float32).astype(np.float64)
     rows, K = v.shape
     assert K % group == 0
     g = v.reshape(rows, K // group, group)
     amax = np.max(np.abs(g), axis=2)
-    s = fp16(fp32(amax / INT4_QMAX))
-    s = np.where(np.isinf(s), 65504.0, s)                    # saturate the scale
-    with np.errstate(divide="ignore"):
-        inv = fp32(np.where(s > 0, 1.0 / np.where(s > 0, s, 1.0), 0.0))
-    y = fp32(g * inv[:, :, None])
-    q = np.clip(np.rint(y), -INT4_QMAX, INT4_QMAX)            # np.rint rounds half to even
-    q = np.where(s[:, :, None] > 0, q, 0.0)
+    s = FP16_GRID[rne_quotient_index(amax, INT4_QMAX, FP16_GRID)]   # products mid * 7: <= 15 bits
+    live = s > 0
+    mag = rne_quotient_index(g, np.where(live, s, 1.0), INT4_GRID)  # products (k + 1/2) s: <= 15 bits
+    q = np.where(np.signbit(g), -mag, mag)
+    q = np.where(live[..., None], q, 0)
     return q.reshape(rows, K).astype(np.int8), s
 
 
@@ -478,30 +536,41 @@ def deltaquant_decode(enc: dict) -> np.ndarray:
     return core[enc["block_of_token"]] + dequantize_nvfp4(enc["delta_codes"], enc["delta_scales"])
 
 
-def fake_quant_int(x: np.ndarray, bits: int, axis=None) -> np.ndarray:
-    """Symmetric uniform quantize-dequantize: s = max|x| / (2^(b-1) - 1) per
-    tensor (or per slice along ``axis``), round half to even, clamp to +-qmax."""
-    qmax = 2 ** (bits - 1) - 1
+# ---------------------------------------------------------------------------
+# The method in real arithmetic with per-tensor integer quantization: the
+# setting of the handbook's printed error tables ([P3] outlier, SmoothQuant and
+# SVDQuant sections). Composed from eq. (1), the smoothing rule and the SVD
+# split above, in fp64 and with no storage format.
+# ---------------------------------------------------------------------------
+
+def int_quant_dequant(t: np.ndarray, bits: int, axis=None) -> np.ndarray:
+    """s * Q(t) of eq. (1) for signed ``bits``-bit integers: one scale
+    s = max|t| / q_max for the whole tensor (axis None) or per slice along
+    ``axis``; Q = round(t / s) half to even, clipped to +-q_max. An all-zero
+    tensor or slice stays zero."""
+    q_max = 2 ** (bits - 1) - 1
+    t = np.asarray(t, dtype=np.float64)
+    amax = np.abs(t).max(axis=axis, keepdims=axis is not None)
+    s = np.where(amax > 0, amax / q_max, 1.0)
+    return s * np.clip(np.rint(t / s), -q_max, q_max)
+
+
+def smoothed_pair(x: np.ndarray, W_io: np.ndarray, alpha: float = 0.5):
+    """(X_hat, W_hat) = (X diag(lambda)^-1, diag(lambda) W) for W_io in the
+    paper's (in x out) orientation, lambda64 of the fp64 channel maxima."""
     x = np.asarray(x, dtype=np.float64)
-    amax = np.max(np.abs(x)) if axis is None else np.max(np.abs(x), axis=axis, keepdims=True)
-    s = np.maximum(amax, 1e-8) / qmax
-    return np.clip(np.rint(x / s), -qmax, qmax) * s
+    W_io = np.asarray(W_io, dtype=np.float64)
+    lam = lambda64(np.abs(x).max(axis=0), np.abs(W_io).max(axis=1), alpha)
+    return x / lam, lam[:, None] * W_io
 
 
-def smooth_fp(x: np.ndarray, W: np.ndarray, alpha: float = 0.5):
-    """X_hat = X / lambda, W_hat = lambda[:, None] * W for W in (in x out)
-    orientation, lambda from the activation and weight channel maxima."""
-    lam = np.max(np.abs(x), axis=0) ** alpha / np.max(np.abs(W), axis=1) ** (1.0 - alpha)
-    return x / lam, W * lam[:, None]
-
-
-def svdquant_fakequant(x: np.ndarray, W: np.ndarray, rank: int, q) -> np.ndarray:
-    """q(X_hat) q(R) + X_hat L1 L2 with L1 = U_r S_r, L2 = V_r^T, R = W_hat - L1 L2."""
-    xs, Ws = smooth_fp(x, W)
-    U, S, Vt = np.linalg.svd(Ws, full_matrices=False)
-    L1, L2 = U[:, :rank] * S[:rank], Vt[:rank]
-    R = Ws - L1 @ L2
-    return q(xs) @ q(R) + xs @ L1 @ L2
+def fakequant_output(x: np.ndarray, W_io: np.ndarray, rank: int, q, alpha: float = 0.5) -> np.ndarray:
+    """Eq. (5) in real arithmetic: X_hat L1 L2 + q(X_hat) q(R) with
+    R = W_hat - L1 L2 (rank 0: q(X_hat) q(W_hat)); ``q`` is a quantize-
+    dequantize function."""
+    xh, Wh = smoothed_pair(x, W_io, alpha)
+    L1, L2, _ = svd_split(Wh, rank)
+    return q(xh) @ q(Wh - L1 @ L2) + (xh @ L1) @ L2
 
 
 # ---------------------------------------------------------------------------

@@ -45,7 +45,7 @@ def test_handbook_outlier_table(handbook):
     for scale, row in tab["outlier_table"]["rows"].items():
         x = base.copy()
         x[:, :4] *= float(scale)
-        got = [O.rel_fro(O.fake_quant_int(x, b, ax)[:, 4:], x[:, 4:])
+        got = [O.rel_fro(O.int_quant_dequant(x, b, ax)[:, 4:], x[:, 4:])
                for b, ax in ((8, None), (8, 0), (4, None), (4, 0))]
         assert [_r4(g) for g in got] == row, scale
 
@@ -56,9 +56,9 @@ def test_handbook_smoothquant_table(handbook):
     x = base.copy()
     x[:, :4] *= 50
     y = x @ W
-    q8 = lambda a: O.fake_quant_int(a, 8)  # noqa: E731
-    q4 = lambda a: O.fake_quant_int(a, 4)  # noqa: E731
-    xs, Ws = O.smooth_fp(x, W)
+    q8 = lambda a: O.int_quant_dequant(a, 8)  # noqa: E731
+    q4 = lambda a: O.int_quant_dequant(a, 4)  # noqa: E731
+    xs, Ws = O.smoothed_pair(x, W)
     assert _r4(O.rel_fro(q8(x) @ q8(W), y)) == t["w8a8"]
     assert _r4(O.rel_fro(q8(xs) @ q8(Ws), y)) == t["w8a8_smooth"]
     assert _r4(O.rel_fro(q4(x) @ q4(W), y)) == t["w4a4"]
@@ -71,14 +71,9 @@ def test_handbook_svdquant_table(handbook):
     x = base.copy()
     x[:, :4] *= 50
     y = x @ W
-    q4 = lambda a: O.fake_quant_int(a, 4)  # noqa: E731
+    q4 = lambda a: O.int_quant_dequant(a, 4)  # noqa: E731
     for r, want in t["rank"].items():
-        r = int(r)
-        if r == 0:
-            xs, Ws = O.smooth_fp(x, W)
-            got = O.rel_fro(q4(xs) @ q4(Ws), y)
-        else:
-            got = O.rel_fro(O.svdquant_fakequant(x, W, r, q4), y)
+        got = O.rel_fro(O.fakequant_output(x, W, int(r), q4), y)
         assert _r4(got) == want, r
     assert _r4(O.rel_fro(q4(base) @ q4(W), base @ W)) == t["no_outlier_w4a4_floor"]
 
@@ -96,7 +91,7 @@ def test_prepare_weights_matches_handbook_flow(handbook):
     P = O.prepare_weights(W_lin, O.channel_amax(x), 0.5, 32)
     lam = P["lam32"].astype(np.float64)
     xs = x / lam
-    q4 = lambda a: O.fake_quant_int(a, 4)  # noqa: E731
+    q4 = lambda a: O.int_quant_dequant(a, 4)  # noqa: E731
     yq = q4(xs) @ q4(P["R32"].astype(np.float64)) + xs @ (lam[:, None] * P["L1p"]) @ P["L2"]
     assert abs(O.rel_fro(yq, y) - tab["svdquant_table"]["rank"]["32"]) < 2e-3
 
@@ -340,7 +335,7 @@ def test_eq7_eq8_gaussian_residual_monte_carlo():
         m_fro = np.mean([O.fro(R) for R in Rs])
         assert m_max <= c * m_fro
         quantizers = {
-            "int4 per tensor": (7, lambda R: O.fake_quant_int(R, 4)),
+            "int4 per tensor": (7, lambda R: O.int_quant_dequant(R, 4)),
             "nvfp4 g16": (6, lambda R: O.dequantize_nvfp4(*O.quantize_nvfp4(R))),
             "int4 g64": (7, lambda R: O.dequantize_int4(*O.quantize_int4(R))),
         }
@@ -349,7 +344,7 @@ def test_eq7_eq8_gaussian_residual_monte_carlo():
             assert m_err <= c * math.sqrt(size) / qmax * m_fro, name
         # uniform rounding: error variance step^2 / 12 per element
         for R in Rs[:4]:
-            err2 = O.fro(R - O.fake_quant_int(R, 4)) ** 2
+            err2 = O.fro(R - O.int_quant_dequant(R, 4)) ** 2
             step = np.abs(R).max() / 7
             assert abs(err2 / (size * step ** 2 / 12) - 1) < 0.05
             _, s = O.quantize_int4(R)
