@@ -49,6 +49,7 @@ METRIC = "SVDQuant W4A4 linear effective TFLOPS (2MNK + 2Mr(K+N)) per layer call
 DEFAULT_WORKLOAD = synth.FLUX_QKV.name
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP4_PER_BF16 = 4.0        # nominal dense FP4 : BF16 tensor throughput ratio on B200 (9 : 2.25 PFLOP/s)
+DATASHEET_FP4_TFLOPS = 9000.0
 
 
 def parse():
@@ -381,6 +382,73 @@ def int4_extras(args, w, step4, X, Y, X_cpu, W_cpu, flops_step, world, rank_id, 
     return e2e, cpu
 
 
+def flux_shape_summary(S, w: synth.Workload, dev, n: int, fp4_peak: float) -> dict:
+    """Layer and GEMM figures of another FLUX projection, timed like the main
+    workload: rotating input sets larger than twice the L2, the layer block with
+    one event pair (dependent launches overlap), the GEMM per launch (events
+    around each kernel) and back to back. Weights are prepared by the library."""
+    X_cpu, W_cpu = synth.generate(w)
+    X, W = X_cpu.to(dev), W_cpu.to(dev)
+    P = S.svdq_prepare_weights(W, S.svdq_channel_amax(X), w.alpha, w.rank)
+    del W
+    set_bytes = X.numel() * 2 + weight_bytes(P)
+    n_sets = max(2, min(16, -(-2 * L2_BYTES // set_bytes)))
+    sets = [(X, P)] + [(X.clone(), clone_weights(P)) for _ in range(n_sets - 1)]
+    Qx = torch.empty(w.M, w.K // 2, dtype=torch.uint8, device=dev)
+    Sx = torch.empty(S.svdq_act_sizes(S.LayerShape(w.M, w.K, w.N, w.rank))[1], dtype=torch.uint8, device=dev)
+    T = torch.empty(w.M, w.rank, dtype=torch.bfloat16, device=dev)
+    Y = torch.empty(w.M, w.N, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def quant(i):
+        X_, P_ = sets[i % n_sets]
+        S.svdq_quantize_act(X_, P_.inv_lam, P_.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
+
+    def gemm(i):
+        S.svdq_linear(Qx, Sx, T, sets[i % n_sets][1], S.SVDQ_FUSED, out=Y)
+
+    def block(fn):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        torch.cuda._sleep(2_000_000)
+        e0.record(stream)
+        for i in range(n):
+            fn(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / n
+
+    for i in range(5):
+        quant(i)
+        gemm(i)
+    layer_ms = block(lambda i: (quant(i), gemm(i)))
+    gemm_block = block(gemm)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    torch.cuda.synchronize()
+    torch.cuda._sleep(2_000_000)
+    for i in range(n):
+        ev[i][0].record(stream)
+        quant(i)
+        ev[i][1].record(stream)
+        gemm(i)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    S.svdq_check()
+    q_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    g_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    g_tf = gemm_flops(w) / (g_ms * 1e-3) / 1e12
+    gb_tf = gemm_flops(w) / (gemm_block * 1e-3) / 1e12
+    return {"workload": w.name, "layer_ms": round(layer_ms, 4),
+            "layer_tflops": round(w.flops() / (layer_ms * 1e-3) / 1e12, 1),
+            "quantize_ms": round(q_ms, 4), "quantize_gbs": round(quantize_bytes(w) / (q_ms * 1e-3) / 1e9, 1),
+            "gemm_ms": round(g_ms, 4), "gemm_tflops": round(g_tf, 1),
+            "gemm_frac": round(g_tf / fp4_peak, 4), "gemm_frac_datasheet_9pf": round(g_tf / DATASHEET_FP4_TFLOPS, 4),
+            "gemm_block_ms": round(gemm_block, 4), "gemm_block_tflops": round(gb_tf, 1),
+            "gemm_block_frac": round(gb_tf / fp4_peak, 4),
+            "gemm_block_frac_datasheet_9pf": round(gb_tf / DATASHEET_FP4_TFLOPS, 4),
+            "fp4_peak_tflops": round(fp4_peak, 1), "input_sets": n_sets}
+
+
 def aggregate_max(value: float, world: int) -> float:
     """Max of a per-rank scalar over all ranks (identity at world size 1)."""
     if world <= 1:
@@ -554,7 +622,11 @@ def run_ours(args):
     value = flops_step * world / (ms_per_step * 1e-3) / 1e12
 
     peaks, peak_src = load_peaks()
-    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
+    # the GEMM is timed alone inside a region of a few ms, so the burst bf16
+    # figure is the matching denominator; the sustained one and the 9 PFLOP/s
+    # datasheet figure are reported beside it
+    fp4_peak = FP4_PER_BF16 * peaks["bf16_tflops"]
+    fp4_sustained = FP4_PER_BF16 * peaks["bf16_tflops_sustained"]
     k2_ms = statistics.mean(k2)
     k1_ms = statistics.mean(k1)
     achieved = gemm_flops(w) / (k2_ms * 1e-3) / 1e12
@@ -568,10 +640,12 @@ def run_ours(args):
     roofline = {"bound": "tensor", "kernel": gemm_kernel_name(w), "achieved": round(achieved, 2),
                 "peak": round(fp4_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4),
                 "traffic": traffic,
-                "peak_note": f"dense FP4 = {FP4_PER_BF16:g} x {peak_src} sustained bf16 "
-                             f"{peaks['bf16_tflops_sustained']:.1f} TFLOP/s; "
-                             f"vs 9000 TFLOP/s datasheet: {achieved / 9000:.4f}; "
-                             f"vs {FP4_PER_BF16:g} x burst bf16: {achieved / (FP4_PER_BF16 * peaks['bf16_tflops']):.4f}"}
+                "frac_datasheet_9pf": round(achieved / DATASHEET_FP4_TFLOPS, 4),
+                "frac_4x_sustained_bf16": round(achieved / fp4_sustained, 4),
+                "peak_note": f"dense FP4 = {FP4_PER_BF16:g} x {peak_src} burst bf16 "
+                             f"{peaks['bf16_tflops']:.1f} TFLOP/s (the kernel is timed alone, per launch); "
+                             f"vs {DATASHEET_FP4_TFLOPS:g} TFLOP/s datasheet: {achieved / DATASHEET_FP4_TFLOPS:.4f}; "
+                             f"vs {FP4_PER_BF16:g} x sustained bf16: {achieved / fp4_sustained:.4f}"}
     if int4:
         roofline = {"bound": "alu", "kernel": "svdq_int4_gemm_kernel", "achieved": round(achieved, 2),
                     "peak": round(alu_peak, 1), "unit": "TFLOP/s", "frac": round(achieved / alu_peak, 4),
@@ -637,6 +711,7 @@ def run_ours(args):
             "rank0_gemm_ms": round(statistics.mean(k2z), 4),
             "gemm_block_ms": round(gemm_block_ms, 4),
             "gemm_block_frac": round(gemm_flops(w) / (gemm_block_ms * 1e-3) / 1e12 / fp4_peak, 4),
+            "gemm_block_frac_datasheet_9pf": round(gemm_flops(w) / (gemm_block_ms * 1e-3) / 1e12 / DATASHEET_FP4_TFLOPS, 4),
             "bf16_cublas_ms": round(statistics.mean(kc), 4),
             "bf16_cublas_tflops": round(2 * w.M * w.N * w.K / (statistics.mean(kc) * 1e-3) / 1e12, 1),
         }
@@ -668,6 +743,10 @@ def run_ours(args):
             "gemm_block_frac_fp8": round(gemm_flops(w) / (int4_gemm_block * 1e-3) / 1e12 / fp8_peak, 4),
             "alu_peak_tflops": round(alu_peak, 1), "fp8_peak_tflops": round(fp8_peak, 1),
         }
+
+        # the other FLUX projections, where the GEMM target is stated
+        extras["other_flux_shapes"] = [flux_shape_summary(S, o, dev, n_x, fp4_peak)
+                                       for o in (synth.FLUX_MLP_UP, synth.FLUX_MLP_DOWN) if o.name != w.name]
 
         # end to end through the public API with host buffers: every step copies
         # its X in from pinned host memory and its Y out to pinned host memory.

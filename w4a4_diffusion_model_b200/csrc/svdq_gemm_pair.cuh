@@ -112,11 +112,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     mbar_init(mma_drain, 1);
     fence_mbar_init();
   }
-  __shared__ float rcp_tbl[QNEXT ? 128 : 1];   // fp32(1/s) per E4M3 byte with the sign bit clear
-  if (QNEXT && threadIdx.x < 128) {
-    const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)threadIdx.x, __NV_E4M3)));
-    rcp_tbl[threadIdx.x] = __frcp_rn(sv);
-  }
+  __shared__ float2 rcp_tbl[QNEXT ? 128 : 1];   // bracket of 1/s per E4M3 byte with the sign bit clear
+  if (QNEXT && threadIdx.x < 128) rcp_tbl[threadIdx.x] = e4m3_recip_bracket(threadIdx.x);
   if (warp == kMmaWarp) {
     tmem_alloc_pair(tmem_slot, kTmemCols);
     tmem_relinquish_pair();

@@ -42,7 +42,7 @@ struct NextQuant {
 // band of Y if asked (through the warp's 128B-swizzled staging box).
 template <int BOXES>
 __device__ __forceinline__ void epilogue_quantize_next(const uint32_t (&p)[32 * BOXES], unsigned char* box,
-                                                       const NextQuant& nq, const float* rcp_tbl, const void* tm_y,
+                                                       const NextQuant& nq, const float2* rcp_tbl, const void* tm_y,
                                                        bool store_y, int row0, int col0, int M, int N, int lane) {
   const int row = row0 + lane;
   const int mpad = (M + 127) & ~127;

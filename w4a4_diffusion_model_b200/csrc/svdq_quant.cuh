@@ -25,9 +25,71 @@ __host__ __device__ __forceinline__ size_t native_scale_offset(int r, int g, int
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// ---------------------------------------------------------------- exact-quotient rounding
+// The codes are round-to-nearest-even images of the EXACT quotient v / s
+// (walkthrough eq. (1): round(X / s)). Multiplying by one rounded reciprocal
+// would not do: it carries up to two fp32 roundings and picks the wrong code
+// when v / s sits on or next to a midpoint of the code grid. Instead each
+// value is multiplied by two reciprocals that bracket 1 / s,
+//   r = fp32(1/s),  lo = fp32(r (1 - 2^-21)),  hi = fp32(r (1 + 2^-21)),
+// for which lo < (1/s)(1 - 2^-22) and hi > (1/s)(1 + 2^-22) (each step errs by
+// at most 2^-24 relative), hence |fp32(v lo)| < |v / s| < |fp32(v hi)| for
+// every fp32 v. Rounding is monotone, so when both products give the same
+// code that code is the exact one. They differ only when a midpoint lies in
+// the bracket (relative width < 2^-19.9, so at most one midpoint, and the two
+// codes are neighbours); then |v| is compared with that midpoint times s,
+// which is exact in fp32 (midpoints carry at most 4 significant bits, scales
+// at most 11), and a tie goes to the even code.
+__device__ __forceinline__ float2 recip_bracket(float s) {
+  const float r = __frcp_rn(s);
+  return make_float2(__fmul_rn(r, 1.0f - 0x1p-21f), __fmul_rn(r, 1.0f + 0x1p-21f));
+}
+
+// Value of the E2M1 magnitude code c (0..7): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+__device__ __forceinline__ float e2m1_value(uint32_t c) {
+  return c >= 2u ? __uint_as_float((((c >> 1) + 126u) << 23) | ((c & 1u) << 22)) : 0.5f * (float)c;
+}
+
+// The exact code of v / s given the codes a (of v lo) and b (of v hi) of its
+// bracket; the sign bit is the products' (kept for values rounding to zero).
+__device__ __forceinline__ uint32_t e2m1_resolve(float v, float s, uint32_t a, uint32_t b) {
+  if (a == b) return a;
+  const uint32_t m = a & 7u;                                            // b & 7 == m + 1
+  const float t = __fmul_rn(0.5f * (e2m1_value(m) + e2m1_value(m + 1u)), s);   // exact
+  const float x = fabsf(v);
+  const uint32_t mag = x > t ? m + 1u : x < t ? m : (m + (m & 1u));
+  return mag | (b & 8u);
+}
+
+// E2M1 byte (element 2i low, 2i+1 high) of a pair scaled by `inv`.
+__device__ __forceinline__ uint32_t e2m1_pair(float2 v, float inv) {
+  return (uint32_t)__nv_cvt_float2_to_fp4x2(make_float2(__fmul_rn(v.x, inv), __fmul_rn(v.y, inv)), __NV_E2M1,
+                                            cudaRoundNearest) & 0xFFu;
+}
+
+// Packed codes of 8 pairs (16 values, one NVFP4 group) given the bracket of
+// 1/s: two 32-bit words, pair i in byte i % 4 of word i / 4. `lo`/`hi` are the
+// codes of the two products; the rare differing nibbles are resolved exactly.
+__device__ __forceinline__ uint2 e2m1_group_exact(const float2 (&v)[8], float s, uint2 lo, uint2 hi) {
+  if (((lo.x ^ hi.x) | (lo.y ^ hi.y)) == 0u) return lo;
+  uint32_t w[2] = {lo.x, lo.y};
+  const uint32_t h[2] = {hi.x, hi.y};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int sh = 8 * (i & 3);
+    const uint32_t a = (w[i >> 2] >> sh) & 0xFFu, b = (h[i >> 2] >> sh) & 0xFFu;
+    if (a == b) continue;
+    const uint32_t byte = e2m1_resolve(v[i].x, s, a & 15u, b & 15u) | (e2m1_resolve(v[i].y, s, a >> 4, b >> 4) << 4);
+    w[i >> 2] = (w[i >> 2] & ~(0xFFu << sh)) | (byte << sh);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 // NVFP4 encoding of 16 fp32 values (one group):
-//   s = E4M3_rne_satfinite(fp32(max|v| / 6)); q_i = E2M1_rne_satfinite(fp32(v_i * fp32(1/s)));
-//   all codes +0 when s decodes to 0. Element 2i lands in the low nibble of byte i.
+//   s = E4M3_rne_satfinite(fp32(max|v| / 6)) (fp32 division then RNE equals
+//   one rounding of the exact quotient: a midpoint times 6 is exact in fp32);
+//   q_i = E2M1_rne_satfinite(v_i / s) of the exact quotient; all codes +0 when
+//   s decodes to 0. Element 2i lands in the low nibble of byte i.
 __device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& codes, uint32_t& sbyte) {
   float amax = 0.f;
 #pragma unroll
@@ -40,15 +102,16 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& code
     codes = make_uint2(0u, 0u);
     return;
   }
-  const float inv = __frcp_rn(sval);
-  uint32_t w[2] = {0u, 0u};
+  const float2 ib = recip_bracket(sval);
+  float2 p[8];
+  uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
 #pragma unroll
   for (int b = 0; b < 8; ++b) {
-    const float2 p = make_float2(__fmul_rn(v[2 * b], inv), __fmul_rn(v[2 * b + 1], inv));
-    const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(p, __NV_E2M1, cudaRoundNearest);
-    w[b >> 2] |= (byte & 0xFFu) << (8 * (b & 3));
+    p[b] = make_float2(v[2 * b], v[2 * b + 1]);
+    lo[b >> 2] |= e2m1_pair(p[b], ib.x) << (8 * (b & 3));
+    hi[b >> 2] |= e2m1_pair(p[b], ib.y) << (8 * (b & 3));
   }
-  codes = make_uint2(w[0], w[1]);
+  codes = e2m1_group_exact(p, sval, make_uint2(lo[0], lo[1]), make_uint2(hi[0], hi[1]));
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -108,9 +108,10 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
 // The NVFP4 recipe of nvfp4_encode16 for one group given as 8 packed bf16
 // pairs and its 16 inverse smoothing factors:
 //   v = fp32(x * inv_lambda); s = E4M3_rne_satfinite(fp32(max|v| / 6));
-//   q = E2M1_rne_satfinite(fp32(v * fp32(1/s))), all +0 when s is 0.
-// fp32(1/s) comes from `rcp_tbl`, indexed by the E4M3 byte of s.
-__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float* rcp_tbl,
+//   q = E2M1_rne_satfinite(v / s) of the exact quotient, all +0 when s is 0.
+// The bracket (lo, hi) of 1/s comes from `rcp_tbl`, indexed by the E4M3 byte
+// of s (recip_bracket of its value).
+__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float2* rcp_tbl,
                                                   uint2& codes, uint32_t& sbyte) {
   float2 v[8];
 #pragma unroll
@@ -128,17 +129,33 @@ __device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float
   m[1] = fmaxf(m[1], m[3]);
   const float amax = fmaxf(m[0], m[1]);
   const uint32_t b = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
-  const float inv = rcp_tbl[b & 0x7Fu];
-  uint32_t lo = 0u, hi = 0u;
+  sbyte = b;
+  if (b == 0u) {
+    codes = make_uint2(0u, 0u);
+    return;
+  }
+  const float2 ib = rcp_tbl[b & 0x7Fu];
+  uint32_t lo[2] = {0u, 0u}, hi[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const uint32_t byte = (uint32_t)__nv_cvt_float2_to_fp4x2(mul2_rn(v[i], make_float2(inv, inv)), __NV_E2M1,
-                                                             cudaRoundNearest) & 0xFFu;
-    if (i < 4) lo |= byte << (8 * i);
-    else hi |= byte << (8 * (i - 4));
+    lo[i >> 2] |= (uint32_t)__nv_cvt_float2_to_fp4x2(mul2_rn(v[i], make_float2(ib.x, ib.x)), __NV_E2M1,
+                                                     cudaRoundNearest) << (8 * (i & 3));
+    hi[i >> 2] |= (uint32_t)__nv_cvt_float2_to_fp4x2(mul2_rn(v[i], make_float2(ib.y, ib.y)), __NV_E2M1,
+                                                     cudaRoundNearest) << (8 * (i & 3));
   }
-  sbyte = b;
-  codes = b != 0u ? make_uint2(lo, hi) : make_uint2(0u, 0u);
+  if (((lo[0] ^ hi[0]) | (lo[1] ^ hi[1])) == 0u) {
+    codes = make_uint2(lo[0], lo[1]);
+    return;
+  }
+  const float sval = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3)));
+  codes = e2m1_group_exact(v, sval, make_uint2(lo[0], lo[1]), make_uint2(hi[0], hi[1]));
+}
+
+// Bracketing reciprocals of every E4M3 scale byte with the sign bit clear
+// (byte 0, a zero scale, is never looked up).
+__device__ __forceinline__ float2 e4m3_recip_bracket(uint32_t byte) {
+  const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
+  return recip_bracket(sv);
 }
 
 // What the quantizing warps produce besides T.
@@ -151,11 +168,24 @@ enum QuantCodec : int {
 // The INT4 recipe (walkthrough eq. (1) with q_max = 7, one fp16 scale per 64
 // elements) for 16 fp32 values a thread holds of a 64-element group; the
 // group's four quarters sit in the four lanes of a quad (lane ^ 1, lane ^ 2):
-//   s = fp16_rne(min(fp32(max|v| / 7), 65504));
-//   q = clamp(rint(fp32(v * fp32(1/s))), -7, 7), all 0 when s is 0.
+//   s = fp16_rne(min(fp32(max|v| / 7), 65504)) (one rounding of the exact
+//   quotient: an fp16 midpoint times 7 is exact in fp32);
+//   q = clamp(RNE(v / s), -7, 7) of the exact quotient, all 0 when s is 0.
+// The quotient is bracketed as for the E2M1 codes (recip_bracket); where the
+// two products round to different integers k and k + 1 (in magnitude), |v| is
+// compared with (k + 1/2) s, exact in fp32 (s has 11 significant bits).
 // Codes are written as the E4M3 bytes of the integers (exact), the form the
 // FP8 tensor-core MMA reads; the scale is returned as its fp32 value.
 // Every lane of the warp must call it (quad shuffles).
+__device__ __forceinline__ float int4_resolve(float v, float s, float qa, float qb) {
+  if (qa == qb) return qa;
+  const float m = fminf(fabsf(qa), fabsf(qb));
+  const float t = __fmul_rn(m + 0.5f, s);   // exact
+  const float x = fabsf(v);
+  const float mag = x > t ? m + 1.f : x < t ? m : (fmodf(m, 2.f) == 0.f ? m : m + 1.f);
+  return copysignf(mag, v);
+}
+
 __device__ __forceinline__ void int4_encode_quarter(const float2 (&v)[8], uint4& codes, float& scale) {
   float amax = 0.f;
 #pragma unroll
@@ -168,14 +198,18 @@ __device__ __forceinline__ void int4_encode_quarter(const float2 (&v)[8], uint4&
     codes = make_uint4(0u, 0u, 0u, 0u);
     return;
   }
-  const float inv = __frcp_rn(s);
+  const float2 ib = recip_bracket(s);
   uint32_t b[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float2 p = mul2_rn(v[i], make_float2(inv, inv));
-    // rint is half-to-even; adding +0 turns a -0 into +0 (code 0 is one byte, 0x00)
-    const float2 qv = make_float2(__fadd_rn(fmaxf(fminf(rintf(p.x), 7.f), -7.f), 0.f),
-                                  __fadd_rn(fmaxf(fminf(rintf(p.y), 7.f), -7.f), 0.f));
+    const float2 pl = mul2_rn(v[i], make_float2(ib.x, ib.x)), ph = mul2_rn(v[i], make_float2(ib.y, ib.y));
+    float qx = rintf(pl.x), qy = rintf(pl.y);   // rint is half-to-even
+    const float hx = rintf(ph.x), hy = rintf(ph.y);
+    if (qx != hx) qx = int4_resolve(v[i].x, s, qx, hx);
+    if (qy != hy) qy = int4_resolve(v[i].y, s, qy, hy);
+    // adding +0 turns a -0 into +0 (code 0 is one byte, 0x00)
+    const float2 qv = make_float2(__fadd_rn(fmaxf(fminf(qx, 7.f), -7.f), 0.f),
+                                  __fadd_rn(fmaxf(fminf(qy, 7.f), -7.f), 0.f));
     b[i] = (uint32_t)__nv_cvt_float2_to_fp8x2(qv, __NV_SATFINITE, __NV_E4M3);
   }
   codes = make_uint4(b[0] | (b[1] << 16), b[2] | (b[3] << 16), b[4] | (b[5] << 16), b[6] | (b[7] << 16));
@@ -204,7 +238,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
   using L = QuantSmem<RANK, BM>;
   constexpr int RG = L::kRowGroups;
   extern __shared__ __align__(1024) unsigned char qsmem_raw[];
-  __shared__ float rcp_tbl[128];
+  __shared__ float2 rcp_tbl[128];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(qsmem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBarOffset);
   uint64_t* empty = full + L::kStages;
@@ -225,10 +259,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
     mbar_init(acc_bar, 1);
     fence_mbar_init();
   }
-  if (CODEC == kCodecNvfp4 && threadIdx.x < 128) {   // fp32(1/s) for every E4M3 byte with the sign bit clear
-    const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)threadIdx.x, __NV_E4M3)));
-    rcp_tbl[threadIdx.x] = __frcp_rn(sv);
-  }
+  if (CODEC == kCodecNvfp4 && threadIdx.x < 128) rcp_tbl[threadIdx.x] = e4m3_recip_bracket(threadIdx.x);
   if (RANK > 0 && warp == L::kMmaWarp) {
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
