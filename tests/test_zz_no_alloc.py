@@ -1,7 +1,9 @@
 """svdq_prepare_weights_static: the weight preparation that runs its device
 SVD in the library's fixed scratch instead of a caller workspace. Called
 through the C ABI and compared with svdq_prepare_weights (caller workspace) on
-the same inputs, for two calls in a row; shapes beyond the scratch are refused.
+the same inputs, for two calls in a row (the second one must leave the
+device's free memory and torch's allocation count unchanged); shapes beyond
+the scratch are refused.
 
 This file is collected last and also passes on its own in a fresh process."""
 import ctypes
@@ -21,7 +23,7 @@ def _p(t):
     return ctypes.c_void_p(t.data_ptr() if t is not None else 0)
 
 
-def _static_prepare(lib, W, amax, alpha, rank):
+def _static_prepare(lib, W, amax, alpha, rank, check_no_alloc=False):
     N, K = W.shape
     qr, sr, l1, l2, _ = S.svdq_weight_sizes(S.LayerShape(0, K, N, rank))
     dev = W.device
@@ -33,17 +35,25 @@ def _static_prepare(lib, W, amax, alpha, rank):
         "lam": torch.empty(K, dtype=torch.float32, device=dev),
         "inv_lam": torch.empty(K, dtype=torch.float32, device=dev),
     }
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated()
     st = lib.svdq_prepare_weights_static(
         S.Shape(0, K, N, rank), _p(W), _p(amax), ctypes.c_float(alpha), 0, _p(out["L1p"]), _p(out["L2t"]),
         _p(out["Qr"]), _p(out["Sr"]), _p(out["lam"]), _p(out["inv_lam"]),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     assert st == 0, lib.svdq_last_error().decode()
     assert lib.svdq_check(ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
+    if check_no_alloc:
+        # after a first call has loaded the kernels, a call takes no device
+        # memory: neither from the driver nor from torch's allocator
+        assert torch.cuda.mem_get_info()[0] == free0
+        assert torch.cuda.memory_allocated() == alloc0
     return out
 
 
 @pytest.mark.parametrize("tmpl,K,N,rank", [(synth.TINY, 512, 512, 16), (synth.FLUX_QKV, 3072, 1024, 32),
-                                           (synth.FLUX_MLP_DOWN, 1536, 384, 48)])
+                                           (synth.FLUX_MLP_DOWN, 1536, 384, 48),
+                                           (synth.FLUX_QKV, 3072, 9216, 32)])   # the full QKV weight
 def test_static_scratch_prepare_matches_workspace_prepare(tmpl, K, N, rank):
     if not torch.cuda.is_available():
         pytest.fail("the gpu tests need a CUDA device")
@@ -57,7 +67,7 @@ def test_static_scratch_prepare_matches_workspace_prepare(tmpl, K, N, rank):
     ref = S.svdq_prepare_weights(Wd, amax, 0.5, rank)
     torch.cuda.synchronize()
     for call in range(2):
-        got = _static_prepare(lib, Wd, amax, 0.5, rank)
+        got = _static_prepare(lib, Wd, amax, 0.5, rank, check_no_alloc=call > 0)
         for name in ("lam", "inv_lam", "Qr", "Sr"):
             assert torch.equal(got[name], getattr(ref, name).reshape(got[name].shape)), (call, name)
         for name in ("L1p", "L2t"):

@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "svdq.h"
@@ -85,6 +86,36 @@ svdq_status check_device() {
   return SVDQ_OK;
 }
 
+// Per-device one-time state (kernel attributes, occupancy queries): a value
+// per device ordinal, computed once under a lock by `init` with that device
+// current and read lock-free afterwards. `init` returns a value > 0, or <= 0
+// for a failure that is not cached (the next call retries).
+constexpr int kMaxDevices = 64;
+
+template <typename F>
+int per_device_once(std::atomic<int> (&cache)[kMaxDevices], int dev, F init) {
+  static std::mutex mu;
+  if (dev < 0 || dev >= kMaxDevices) return init();
+  const int v = cache[dev].load(std::memory_order_acquire);
+  if (v > 0) return v;
+  std::lock_guard<std::mutex> lk(mu);
+  int w = cache[dev].load(std::memory_order_relaxed);
+  if (w <= 0) {
+    w = init();
+    if (w > 0) cache[dev].store(w, std::memory_order_release);
+  }
+  return w;
+}
+
+int current_device() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
 // ---------------------------------------------------------------- tensor maps
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -143,14 +174,17 @@ size_t scale_bytes(int64_t rows, int64_t K) { return (size_t)((rows + 127) / 128
 
 // ---------------------------------------------------------------- launchers
 int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
-  if (dev < 64 && cached[dev]) return cached[dev];
-  int n = 148;
-  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 148;
-  if (dev < 64) cached[dev] = n;
-  return n;
+  static std::atomic<int> cache[kMaxDevices];
+  const int dev = current_device();
+  const int n = per_device_once(cache, dev, [dev] {
+    int v = 0;
+    if (dev < 0 || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    return v;
+  });
+  return n > 0 ? n : 148;
 }
 
 // Quantization: one CTA per BM rows (128 or 64) and K slice, one CTA per SM.
@@ -164,21 +198,23 @@ struct QuantLaunch {
   static constexpr auto kern = svdq::quantize_tma_kernel<RANK, BM, CODEC>;
 
   static svdq_status prepare() {   // once per device
-    static bool done[64];
-    int dev = 0;
-    SVDQ_CUDA(cudaGetDevice(&dev));
-    if (dev >= 64 || !done[dev]) {
-      SVDQ_CUDA(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes));
-      if (dev < 64) done[dev] = true;
-    }
+    static std::atomic<int> done[kMaxDevices];
+    cudaError_t err = cudaSuccess;
+    per_device_once(done, current_device(), [&err] {
+      err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kBytes);
+      return err == cudaSuccess ? 1 : 0;
+    });
+    if (err != cudaSuccess)
+      return fail(SVDQ_ERR_CUDA, "cudaFuncSetAttribute(quantize_tma_kernel): %s", cudaGetErrorString(err));
     return SVDQ_OK;
   }
 
-  // Clusters of k CTAs that can be resident at once (cached per k).
+  // Clusters of k CTAs that can be resident at once, per device and k (cached
+  // as count + 1, so that a device where none fit is cached too).
   static int max_clusters(int k) {
-    static int cache[4] = {-1, -1, -1, -1};
-    const int i = k == 2 ? 1 : k == 4 ? 2 : 3;
-    if (cache[i] < 0) {
+    static std::atomic<int> cache[3][kMaxDevices];
+    const int i = k == 2 ? 0 : k == 4 ? 1 : 2;
+    return per_device_once(cache[i], current_device(), [k] {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -193,9 +229,8 @@ struct QuantLaunch {
       int n = 0;
       if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
       cudaGetLastError();
-      cache[i] = n;
-    }
-    return cache[i];
+      return n + 1;
+    }) - 1;
   }
 
   // Largest K split (8, 4, 2, 1) that keeps the grid in one wave; returns the
@@ -349,25 +384,24 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
 // cached per device; also sets the kernel's shared-memory attribute there.
 template <int NB, bool QNEXT = false>
 int pair_clusters() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev < 64 && cached[dev]) return cached[dev];
-  auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB>::kBytes) !=
-      cudaSuccess) {
-    cudaGetLastError();
-    return 0;
-  }
-  cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, attr, false);
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    n = 0;
-  }
-  if (dev < 64) cached[dev] = n;
-  return n;
+  static std::atomic<int> cache[kMaxDevices];
+  // cached as count + 1; a failed attribute call is not cached
+  return per_device_once(cache, current_device(), [] {
+    auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB>::kBytes) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return 0;
+    }
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, attr, false);
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    return n + 1;
+  }) - 1;
 }
 
 template <int NB, bool QNEXT = false>
@@ -506,17 +540,18 @@ svdq_status launch_svd(const svdq_shape& s, const void* W, const float* lam, voi
   float* T2 = reinterpret_cast<float*>(ws + p.off_t2);
   const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(W);
   {
-    static bool done[64];
-    int dev = 0;
-    SVDQ_CUDA(cudaGetDevice(&dev));
-    if (dev >= 64 || !done[dev]) {
+    static std::atomic<int> done[kMaxDevices];
+    cudaError_t err = cudaSuccess;
+    per_device_once(done, current_device(), [&err] {
       const int big = (int)jacobi_smem_bytes(kSvdMaxL), ab = (int)apply_smem_bytes(kSvdMaxL, kSvdMaxL);
-      SVDQ_CUDA(cudaFuncSetAttribute(svd_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big));
-      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
-      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyL1p>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
-      SVDQ_CUDA(cudaFuncSetAttribute(svd_apply_kernel<kApplyL2t>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab));
-      if (dev < 64) done[dev] = true;
-    }
+      if ((err = cudaFuncSetAttribute(svd_jacobi_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, big)) ||
+          (err = cudaFuncSetAttribute(svd_apply_kernel<kApplyF32>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab)) ||
+          (err = cudaFuncSetAttribute(svd_apply_kernel<kApplyL1p>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab)) ||
+          (err = cudaFuncSetAttribute(svd_apply_kernel<kApplyL2t>, cudaFuncAttributeMaxDynamicSharedMemorySize, ab)))
+        return 0;
+      return 1;
+    });
+    if (err != cudaSuccess) return fail(SVDQ_ERR_CUDA, "cudaFuncSetAttribute(svd kernels): %s", cudaGetErrorString(err));
   }
   auto grid_for = [](size_t n) { return (unsigned)((n + 255) / 256 < 2048 ? (n + 255) / 256 : 2048); };
   auto eig_of_gram = [&](const float* buf, int rows, int parts) -> svdq_status {

@@ -253,10 +253,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       uint32_t sfbuf = 0;        // item index mod 2 (scale buffers used in turn)
       bool ready = false;        // the current item's stage and scales are known to be in place
       for (int tile = cluster; tile < ntiles && ok; tile += nclusters, ++tcount) {
-        // CTA-scope waits: the remote arrivals on acc_empty and sf_ready are
-        // relaxed and announce work already completed by its own mechanism
-        // (tcgen05.wait::ld / tcgen05.wait::st), so a cluster-scope acquire
-        // would order nothing and only costs issue time
+        // acc_empty and sf_ready count arrivals from both CTAs, each announcing
+        // TMEM reads / writes that a tcgen05.wait already completed (see
+        // mbar_arrive_remote); the waits take CTA-scope acquire and are
+        // followed by tcgen05.fence::after_thread_sync before the MMAs
         if (!mbar_wait(acc_empty, (tcount & 1u) ^ 1u, kDevErrTimeoutAccum)) {
           ok = false;
           break;
