@@ -490,8 +490,9 @@ def layer_reference_int4(X, W_lin, alpha: float, rank: int, act_amax=None) -> di
 #   * tokens of a video latent [F][H][Wd] are rows in frame, row, column
 #     order; blocks are bf x bh x bw tokens (default 2 x 2 x 2), tiled from
 #     the origin; blocks at a ragged edge hold the tokens that exist;
-#   * core = E4M3_RNE_satfinite of the block's exact mean (fp64), per channel,
-#     with no scale (the page names FP8 and nothing else);
+#   * core = E4M3_RNE_satfinite of the block's exact mean (the fp64 sum of its
+#     tokens in token order, divided by the token count, rounded once), per
+#     channel, with no scale (the page names FP8 and nothing else);
 #   * delta = fp32(x - decode(core)), i.e. relative to the stored core, so
 #     the core's rounding is absorbed by the delta; deltas are NVFP4 (groups of
 #     16 channels, the codec above);
@@ -524,7 +525,10 @@ def deltaquant_encode(X: np.ndarray, dims, block=(2, 2, 2)) -> dict:
     sums = np.zeros((nb, X.shape[1]))
     np.add.at(sums, blk, X)
     counts = np.bincount(blk, minlength=nb).astype(np.float64)
-    core_codes = e4m3_encode_signed(sums / counts[:, None])
+    # E4M3 RNE (satfinite) of the exact quotient sum / count; a negative mean
+    # that rounds to zero keeps the sign bit, a zero sum encodes +0
+    mag = rne_quotient_index(sums, counts, E4M3_GRID)
+    core_codes = (mag | np.where(np.signbit(sums) & (sums != 0), 0x80, 0)).astype(np.uint8)
     core = e4m3_decode(core_codes)
     delta = fp32(X - core[blk])
     codes, scales = quantize_nvfp4(delta)

@@ -99,3 +99,24 @@ def test_smooth_video_premise():
     c, s = O.quantize_nvfp4(N.astype(np.float32))
     err_fp4_n = O.rel_fro(O.dequantize_nvfp4(c, s), N)
     assert err_dq_n > 0.8 * err_fp4_n
+
+
+def test_core_rounds_the_exact_mean_ties_and_double_rounding_cases():
+    """The core is one RNE rounding of the exact block mean: a mean exactly on
+    an E4M3 midpoint goes to the even code; a mean a hair above it (2^-28
+    relative, lost if the mean were first rounded to fp32) goes up; a mean
+    above 448 saturates; a negative mean that rounds to zero keeps the sign."""
+    F, H, Wd, C = 2, 2, 2, 16
+    X = np.zeros((8, C))
+    X[0, 0] = 8.5                      # mean 1.0625: midpoint of 1.0 and 1.125 -> even code 1.0
+    X[0, 1], X[3, 1] = 8.5, 2.0 ** -25  # mean 1.0625 + 2^-28 -> 1.125
+    X[:, 2] = 500.0                    # mean 500 -> 448
+    X[5, 3] = -(2.0 ** -14)            # mean -2^-17 rounds to -0
+    X[:, 4] = -3.0                     # block-constant
+    X[0, 5], X[1, 5] = 1.0, -1.0       # zero sum -> +0
+    assert np.array_equal(O.bf16(X), X)
+    enc = O.deltaquant_encode(X, (F, H, Wd))
+    core = enc["core_codes"][0]
+    assert O.e4m3_decode(core[0]) == 1.0 and O.e4m3_decode(core[1]) == 1.125
+    assert O.e4m3_decode(core[2]) == 448.0 and core[3] == 0x80 and O.e4m3_decode(core[4]) == -3.0
+    assert core[5] == 0x00
