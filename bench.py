@@ -449,6 +449,43 @@ def flux_shape_summary(S, w: synth.Workload, dev, n: int, fp4_peak: float) -> di
             "fp4_peak_tflops": round(fp4_peak, 1), "input_sets": n_sets}
 
 
+def deltaquant_bytes(F: int, H: int, W: int, C: int) -> int:
+    """Algorithmic HBM bytes of one DeltaQuant encode: read the bf16 tokens;
+    write the E4M3 cores, the packed delta codes and their native scales."""
+    T = F * H * W
+    blocks = ((F + 1) // 2) * ((H + 1) // 2) * ((W + 1) // 2)
+    return 2 * T * C + blocks * C + T * C // 2 + (T + 127) // 128 * (C // 64) * 512
+
+
+def deltaquant_summary(S, dev, n: int, dims=(16, 32, 48), C: int = 3072) -> dict:
+    """The DeltaQuant encoder on a video latent (smooth synthetic tokens),
+    launched back to back over two copies of the input (more than twice the
+    L2) with one event pair around the block."""
+    F, H, W = dims
+    X0 = synth.smooth_video(F, H, W, C, seed=77).to(dev)
+    Xs = [X0, X0.clone()]
+    cb, _, sb = S.svdq_deltaquant_sizes(F, H, W, C)
+    out = (torch.empty(cb // C, C, dtype=torch.uint8, device=dev),
+           torch.empty(F * H * W, C // 2, dtype=torch.uint8, device=dev),
+           torch.empty(sb, dtype=torch.uint8, device=dev))
+    for i in range(3):
+        S.svdq_deltaquant_encode(Xs[i % 2], dims, out=out)
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(2_000_000)
+    e0.record(stream)
+    for i in range(n):
+        S.svdq_deltaquant_encode(Xs[i % 2], dims, out=out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    S.svdq_check()
+    ms = e0.elapsed_time(e1) / n
+    nbytes = deltaquant_bytes(F, H, W, C)
+    return {"kernel": "deltaquant_encode_kernel", "video": f"{F}x{H}x{W} tokens x {C} channels, 2x2x2 blocks",
+            "ms": round(ms, 4), "algorithmic_bytes": nbytes, "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1)}
+
+
 def aggregate_max(value: float, world: int) -> float:
     """Max of a per-rank scalar over all ranks (identity at world size 1)."""
     if world <= 1:
@@ -747,6 +784,9 @@ def run_ours(args):
         # the other FLUX projections, where the GEMM target is stated
         extras["other_flux_shapes"] = [flux_shape_summary(S, o, dev, n_x, fp4_peak)
                                        for o in (synth.FLUX_MLP_UP, synth.FLUX_MLP_DOWN) if o.name != w.name]
+
+        extras["deltaquant"] = deltaquant_summary(S, dev, n_x)
+        extras["deltaquant"]["frac_hbm"] = round(extras["deltaquant"]["gbs"] / peaks["hbm_gbs"], 4)
 
         # end to end through the public API with host buffers: every step copies
         # its X in from pinned host memory and its Y out to pinned host memory.

@@ -283,6 +283,33 @@ SVDQ_API svdq_status svdq_int4_quantize_act(svdq_shape shape, const void* X, con
 SVDQ_API svdq_status svdq_int4_linear(svdq_shape shape, const void* Qx, const void* Sx, const void* T,
                                       const void* Qr, const void* Sr, const void* L2t, void* Y, void* stream);
 
+/* ---------------------------------------------------------------- DeltaQuant
+ * Core + delta encoding of video activations (libaedu.com article on 4-bit
+ * diffusion-model quantization, DeltaQuant paragraphs: tokens of a local 3-D
+ * spatio-temporal block share a core token, their mean, kept in FP8; each
+ * token's difference to it is quantized to 4 bits). The article gives the
+ * method in outline only; the readings here:
+ *   X        bf16 [F*H*W][C]: the tokens of an F-frame, H x W video latent in
+ *            frame, row, column order; C % 64 == 0.
+ *   blocks   2 x 2 x 2 tokens tiled from the origin, numbered in (frame, row,
+ *            column) order of the block grid ceil(F/2) x ceil(H/2) x ceil(W/2);
+ *            blocks at a ragged edge hold the tokens that exist.
+ *   core     uint8 [blocks][C]: E4M3 (fn, saturating at 448) of the block's
+ *            exact mean per channel, rounded once to nearest even; a negative
+ *            mean rounding to zero keeps the sign bit (0x80), a zero sum is 0x00.
+ *   Qd, Sd   the NVFP4 codes [F*H*W][C/2] and native-layout scales of the
+ *            deltas fp32(x - core), grouped by 16 channels, in the format of
+ *            svdq_quantize_act's Qx / Sx (rows past the last token of the last
+ *            128-row scale atom hold zero).
+ * Sizes of the three outputs from svdq_deltaquant_sizes. Shapes: F, H, W >= 1,
+ * F*H*W < 2^31, 64 <= C <= 2^20 with C % 64 == 0; otherwise
+ * SVDQ_ERR_UNSUPPORTED_SHAPE. Pointers as everywhere (device, 16-byte aligned,
+ * caller-owned). Async on stream. */
+SVDQ_API svdq_status svdq_deltaquant_sizes(int64_t F, int64_t H, int64_t W, int64_t C, size_t* core_bytes,
+                                           size_t* qd_bytes, size_t* sd_bytes);
+SVDQ_API svdq_status svdq_deltaquant_encode(int64_t F, int64_t H, int64_t W, int64_t C, const void* X, void* core,
+                                            void* Qd, void* Sd, void* stream);
+
 /* Diagnostic of the failure path (the pages have no counterpart): one thread
  * waits, with the library's bounded wait, on a barrier phase that nothing
  * completes; after the wait limit (2 s) it records the device error word and

@@ -493,9 +493,10 @@ def layer_reference_int4(X, W_lin, alpha: float, rank: int, act_amax=None) -> di
 #   * core = E4M3_RNE_satfinite of the block's exact mean (the fp64 sum of its
 #     tokens in token order, divided by the token count, rounded once), per
 #     channel, with no scale (the page names FP8 and nothing else);
-#   * delta = fp32(x - decode(core)), i.e. relative to the stored core, so
-#     the core's rounding is absorbed by the delta; deltas are NVFP4 (groups of
-#     16 channels, the codec above);
+#   * delta = fp32(x - decode(core)), the exact difference rounded once to
+#     fp32, i.e. relative to the stored core, so the core's rounding is
+#     absorbed by the delta; deltas are NVFP4 (groups of 16 channels, the codec
+#     above);
 #   * reconstruction x~ = decode(core) + deq(delta).
 # Oracle only: no kernel consumes this encoding yet.
 
@@ -530,7 +531,8 @@ def deltaquant_encode(X: np.ndarray, dims, block=(2, 2, 2)) -> dict:
     mag = rne_quotient_index(sums, counts, E4M3_GRID)
     core_codes = (mag | np.where(np.signbit(sums) & (sums != 0), 0x80, 0)).astype(np.uint8)
     core = e4m3_decode(core_codes)
-    delta = fp32(X - core[blk])
+    # one rounding of the exact difference (bf16 and E4M3 values are exact in fp32)
+    delta = X.astype(np.float32) - core[blk].astype(np.float32)
     codes, scales = quantize_nvfp4(delta)
     return dict(block_of_token=blk, core_codes=core_codes, delta_codes=codes, delta_scales=scales)
 

@@ -172,3 +172,15 @@ def test_int4_sizes_and_argument_checks(lib):
         sh0 = S.Shape(128, 256, 128, 0)
         assert lib.svdq_int4_linear(sh0, good, good, None, good, good, None, good, None) == 5
         assert lib.svdq_int4_quantize_residual(sh0, good, good, None, None, good, good, None) == 5
+
+
+def test_deltaquant_sizes_and_argument_checks(lib):
+    core, qd, sd = S.svdq_deltaquant_sizes(5, 7, 9, 192)      # 3 x 4 x 5 blocks, 315 tokens
+    assert core == 60 * 192 and qd == 315 * 96 and sd == 3 * 3 * 512
+    for F, H, W, C in ((0, 4, 4, 64), (2, 2, 2, 48), (2, 2, 2, 0), (2, 2, 2, (1 << 20) + 64), (1 << 20, 1 << 11, 1, 64)):
+        a = ctypes.c_size_t()
+        assert lib.svdq_deltaquant_sizes(F, H, W, C, ctypes.byref(a), None, None) == 2, (F, H, W, C)
+    good, bad = ctypes.c_void_p(1 << 20), ctypes.c_void_p((1 << 20) + 8)
+    assert lib.svdq_deltaquant_encode(2, 2, 2, 64, None, good, good, good, None) == 1
+    assert lib.svdq_deltaquant_encode(2, 2, 2, 64, good, good, bad, good, None) == 3
+    assert lib.svdq_deltaquant_encode(2, 2, 2, 96, good, good, good, good, None) == 2

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "svdq.h"
+#include "svdq_deltaquant.cuh"
 #include "svdq_gemm.cuh"
 #include "svdq_gemm_pair.cuh"
 #include "svdq_int4.cuh"
@@ -1006,6 +1007,58 @@ svdq_status svdq_int4_linear(svdq_shape s, const void* Qx, const void* Sx, const
     if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
   if ((r = check_device()) != SVDQ_OK) return r;
   return launch_int4_gemm(s, Qx, Sx, T, Qr, Sr, L2t, Y, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+svdq_status check_video_shape(int64_t F, int64_t H, int64_t W, int64_t C) {
+  if (F < 1 || H < 1 || W < 1 || C < 64 || C % 64 || C > (1ll << 20) || F > (1ll << 31) || H > (1ll << 31) ||
+      W > (1ll << 31) || F * H > (1ll << 31) || F * H * W > (1ll << 31) - 1)
+    return fail(SVDQ_ERR_UNSUPPORTED_SHAPE,
+                "video F=%lld H=%lld W=%lld C=%lld: need F, H, W >= 1, F*H*W < 2^31, C a multiple of 64 in [64, 2^20]",
+                (long long)F, (long long)H, (long long)W, (long long)C);
+  return SVDQ_OK;
+}
+
+int64_t video_blocks(int64_t F, int64_t H, int64_t W) { return ((F + 1) / 2) * ((H + 1) / 2) * ((W + 1) / 2); }
+
+}  // namespace
+
+svdq_status svdq_deltaquant_sizes(int64_t F, int64_t H, int64_t W, int64_t C, size_t* core_bytes, size_t* qd_bytes,
+                                  size_t* sd_bytes) {
+  g_last_error[0] = 0;
+  svdq_status r = check_video_shape(F, H, W, C);
+  if (r != SVDQ_OK) return r;
+  const int64_t tokens = F * H * W;
+  if (core_bytes) *core_bytes = (size_t)video_blocks(F, H, W) * (size_t)C;
+  if (qd_bytes) *qd_bytes = (size_t)tokens * (size_t)(C / 2);
+  if (sd_bytes) *sd_bytes = scale_bytes(tokens, C);
+  return SVDQ_OK;
+}
+
+svdq_status svdq_deltaquant_encode(int64_t F, int64_t H, int64_t W, int64_t C, const void* X, void* core, void* Qd,
+                                   void* Sd, void* stream) {
+  g_last_error[0] = 0;
+  svdq_status r = check_video_shape(F, H, W, C);
+  if (r != SVDQ_OK) return r;
+  if (!X || !core || !Qd || !Sd) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
+  const void* ptrs[] = {X, core, Qd, Sd};
+  for (const void* p : ptrs)
+    if (!aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
+  if ((r = check_device()) != SVDQ_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t tokens = F * H * W;
+  if (tokens % 128) {   // zero the last scale atom row block; the kernel writes its live rows
+    const size_t atoms = (size_t)(C / 64) * 512u;
+    SVDQ_CUDA(cudaMemsetAsync(static_cast<uint8_t*>(Sd) + (size_t)(tokens / 128) * atoms, 0, atoms, st));
+  }
+  const dim3 grid((unsigned)video_blocks(F, H, W),
+                  (unsigned)((C / 16 + svdq::kDqGroupsPerCta - 1) / svdq::kDqGroupsPerCta));
+  svdq::deltaquant_encode_kernel<<<grid, svdq::kDqThreads, 0, st>>>(
+      static_cast<const __nv_bfloat16*>(X), static_cast<uint8_t*>(core), static_cast<uint8_t*>(Qd),
+      static_cast<uint8_t*>(Sd), (int)F, (int)H, (int)W, (int)C);
+  SVDQ_LAUNCHED("deltaquant_encode_kernel");
+  return SVDQ_OK;
 }
 
 svdq_status svdq_selftest_timeout(void* stream) {

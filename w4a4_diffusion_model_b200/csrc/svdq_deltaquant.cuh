@@ -1,0 +1,161 @@
+// DeltaQuant-style core + delta encoding of video activations (libaedu.com
+// article on 4-bit diffusion-model quantization, DeltaQuant paragraphs: the
+// tokens of a local 3-D spatio-temporal block share a core token, their mean,
+// kept in FP8; each token's difference to it is quantized to 4 bits).
+//
+// Tokens are rows of X [F*H*W][C] bf16 in frame, row, column order; blocks are
+// 2 x 2 x 2 tokens tiled from the origin, edge blocks holding the tokens that
+// exist (n = 1, 2, 4 or 8 of them). Per block b and channel c:
+//   core[b][c] = E4M3_RNE_satfinite(sum / n) of the exact sum of the block's
+//                tokens, rounded once; a negative mean rounding to zero keeps
+//                the sign bit, a zero sum encodes +0;
+//   delta[t][c] = fp32(x[t][c] - decode(core[b][c])), the exact difference
+//                rounded once (one fp32 subtraction: both operands are fp32
+//                values), NVFP4-encoded along C with the library's codec
+//                (nvfp4_encode16: E4M3 scale of amax / 6, E2M1 codes of the
+//                exact quotients), codes packed two per byte, scales in the
+//                native tile layout of the 4-bit GEMM.
+//
+// The exact sum. Eight bf16 values carry 8-bit significands; when the nonzero
+// ones span at most 13 binades (max|x| <= 2^13 min|x|) their sum needs at most
+// 8 + 13 + 3 = 24 bits and the fp32 additions are exact, and so is the mean
+// (n is a power of two): the hardware fp32 -> E4M3 conversion then rounds the
+// exact mean once. A channel whose values span more binades (or whose values
+// reach 2^124, where eight of them could overflow fp32) takes the fp64 path:
+// the sum in token order, exact for spreads up to ~45 binades and otherwise
+// the same fp64 additions the reference makes, rounded to E4M3 from fp64.
+//
+// A CTA of 128 threads handles one block and up to 64 16-channel groups
+// (grid: x = block, y = 1024-channel chunk); two lanes share a group, 8
+// channels each, so that a warp reads each token row as one coalesced 512-byte
+// span. A lane forms its 8 sums and cores, then encodes each token's deltas
+// with the pair recipe nvfp4_encode8_pair; the 8 lanes of 4 consecutive groups
+// pool their scale bytes into one 32-bit store. Rows of the last 128-row scale
+// atom past the last token are zeroed by the host before the launch.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "svdq_quant.cuh"
+
+namespace svdq {
+
+__device__ __forceinline__ float e4m3_to_float(uint32_t byte) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
+}
+
+constexpr int kDqThreads = 128;
+constexpr int kDqGroupsPerCta = kDqThreads / 2;
+
+__global__ void __launch_bounds__(kDqThreads) deltaquant_encode_kernel(const __nv_bfloat16* __restrict__ X,
+                                                                       uint8_t* __restrict__ core,
+                                                                       uint8_t* __restrict__ Qd,
+                                                                       uint8_t* __restrict__ Sd, int F, int H, int W,
+                                                                       int C) {
+  const int G = C >> 4;                                   // 16-channel groups per token (a multiple of 4)
+  const int nbh = (H + 1) >> 1, nbw = (W + 1) >> 1;
+  const int b = blockIdx.x;                               // the block
+  const int bw = b % nbw, bh = (b / nbw) % nbh, bf = b / (nbw * nbh);
+  const int gl = blockIdx.y * kDqGroupsPerCta + (threadIdx.x >> 1);
+  const bool live = gl < G;                               // lanes past C (whole quads of groups) store nothing
+  const int g = live ? gl : G - 4 + ((threadIdx.x >> 1) & 3);
+  const int half = threadIdx.x & 1;
+  const int c0 = 16 * g + 8 * half;                       // this lane's 8 channels
+
+  // the block's tokens in token order (frame, row, column)
+  int rows[8];
+  int n = 0, present = 0;
+#pragma unroll
+  for (int df = 0; df < 2; ++df)
+#pragma unroll
+    for (int dh = 0; dh < 2; ++dh)
+#pragma unroll
+      for (int dw = 0; dw < 2; ++dw) {
+        const int f = 2 * bf + df, h = 2 * bh + dh, w = 2 * bw + dw;
+        const int t = 4 * df + 2 * dh + dw;
+        const bool ok = f < F && h < H && w < W;
+        rows[t] = ok ? (f * H + h) * W + w : -1;
+        n += ok;
+        present |= ok ? 1 << t : 0;
+      }
+  uint32_t xw[32];                                        // token t, pair i at xw[4 t + i]
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    uint4 a = make_uint4(0u, 0u, 0u, 0u);
+    if (rows[t] >= 0) a = __ldg(reinterpret_cast<const uint4*>(X + (size_t)rows[t] * C + c0));
+    xw[4 * t + 0] = a.x; xw[4 * t + 1] = a.y; xw[4 * t + 2] = a.z; xw[4 * t + 3] = a.w;
+  }
+  // fp32 sums (exact when the spread test below passes), |x| max and nonzero
+  // |x| min per channel; missing tokens hold +0 and change none of them
+  float sum[8], mx[8];
+  uint32_t mn[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sum[i] = 0.f;
+    mx[i] = 0.f;
+    mn[i] = 0xFFFFFFFFu;
+  }
+#pragma unroll
+  for (int t = 0; t < 8; ++t)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const uint32_t w = xw[4 * t + (i >> 1)];
+      const uint32_t u = (i & 1) ? (w & 0xFFFF0000u) : (w << 16);
+      sum[i] = __fadd_rn(sum[i], __uint_as_float(u));
+      mx[i] = fmaxf(mx[i], fabsf(__uint_as_float(u)));
+      mn[i] = min(mn[i], (u & 0x7FFFFFFFu) - 1u);         // a zero wraps to the maximum
+    }
+  const float inv_n = 1.0f / (float)n;                    // n is 1, 2, 4 or 8: exact
+  float cval[8];
+  uint32_t cb[2] = {0u, 0u};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float mnf = __uint_as_float(mn[i] + 1u);        // +0 when every value is zero
+    const bool exact = mx[i] < 0x1p124f && (mn[i] == 0xFFFFFFFFu || mx[i] <= mnf * 8192.0f);
+    uint32_t byte;
+    if (exact) {
+      const float mean = sum[i] * inv_n;
+      byte = mean == 0.f ? 0u : (uint32_t)__nv_cvt_float_to_fp8(mean, __NV_SATFINITE, __NV_E4M3);
+    } else {   // wide range: the fp64 sum in token order (i and t are compile-time: registers only)
+      double sd = 0.0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (!(present & (1 << t))) continue;
+        const uint32_t w = xw[4 * t + (i >> 1)];
+        sd += (double)((i & 1) ? bf16hi(w) : bf16lo(w));
+      }
+      byte = sd == 0.0 ? 0u : (uint32_t)__nv_cvt_double_to_fp8(sd / (double)n, __NV_SATFINITE, __NV_E4M3);
+    }
+    cval[i] = e4m3_to_float(byte);
+    cb[i >> 2] |= byte << (8 * (i & 3));
+  }
+  if (live) *reinterpret_cast<uint2*>(core + (size_t)b * C + c0) = make_uint2(cb[0], cb[1]);
+
+  // Every lane runs all eight token positions (edge blocks lack some tokens):
+  // the shuffles are taken by the whole warp, only the stores depend on the
+  // token existing.
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    float d[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = xw[4 * t + i];
+      d[2 * i] = __fsub_rn(bf16lo(w), cval[2 * i]);
+      d[2 * i + 1] = __fsub_rn(bf16hi(w), cval[2 * i + 1]);
+    }
+    uint32_t codes, sb;
+    nvfp4_encode8_pair(d, codes, sb);
+    // lanes 8j, 8j+2, 8j+4, 8j+6 hold the scales of groups 4j'..4j'+3
+    const uint32_t s1 = __shfl_sync(0xFFFFFFFFu, sb, (lane + 2) & 31), s2 = __shfl_sync(0xFFFFFFFFu, sb, (lane + 4) & 31),
+                   s3 = __shfl_sync(0xFFFFFFFFu, sb, (lane + 6) & 31);
+    if (!live || rows[t] < 0) continue;
+    const size_t row = (size_t)rows[t];
+    *reinterpret_cast<uint32_t*>(Qd + row * (size_t)(C >> 1) + (c0 >> 1)) = codes;
+    if ((lane & 7) == 0)
+      *reinterpret_cast<uint32_t*>(Sd + native_scale_offset(rows[t], g, C)) = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
+}  // namespace svdq

@@ -114,6 +114,37 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& code
   codes = e2m1_group_exact(p, sval, make_uint2(lo[0], lo[1]), make_uint2(hi[0], hi[1]));
 }
 
+// The same NVFP4 recipe for a group of 16 held by two lanes (lane ^ 1), 8
+// values each: the group's amax is pooled with one shuffle, both lanes derive
+// the same scale, and each lane returns the packed codes of its own 8 values
+// (one 32-bit word: element 2i in the low nibble of byte i). Every lane of the
+// warp must call it.
+__device__ __forceinline__ void nvfp4_encode8_pair(const float (&v)[8], uint32_t& codes, uint32_t& sbyte) {
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
+  const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+  const float sval = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
+  sbyte = (uint32_t)sb;
+  if (sval == 0.f) {
+    codes = 0u;
+    return;
+  }
+  const float2 ib = recip_bracket(sval);
+  uint32_t lo = 0u, hi = 0u;
+  float2 p[8];
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    p[b] = make_float2(v[2 * b], v[2 * b + 1]);
+    lo |= e2m1_pair(p[b], ib.x) << (8 * b);
+    hi |= e2m1_pair(p[b], ib.y) << (8 * b);
+  }
+#pragma unroll
+  for (int b = 4; b < 8; ++b) p[b] = make_float2(0.f, 0.f);
+  codes = e2m1_group_exact(p, sval, make_uint2(lo, 0u), make_uint2(hi, 0u)).x;
+}
+
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                                uint32_t b0, uint32_t b1) {
   asm volatile(

@@ -33,7 +33,7 @@ EXPORTS = [
     "svdq_linear", "svdq_linear_quantize_next", "svdq_linear_quantize_next_workspace", "svdq_append_lowrank",
     "svdq_selftest_timeout", "svdq_scales_to_canonical", "svdq_check",
     "svdq_int4_act_sizes", "svdq_int4_weight_sizes", "svdq_int4_quantize_residual", "svdq_int4_quantize_act",
-    "svdq_int4_linear",
+    "svdq_int4_linear", "svdq_deltaquant_sizes", "svdq_deltaquant_encode",
 ]
 
 
@@ -94,6 +94,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_int4_quantize_residual.restype = st
     lib.svdq_int4_quantize_act.argtypes, lib.svdq_int4_quantize_act.restype = [Shape, vp, vp, vp, vp, vp, vp, vp], st
     lib.svdq_int4_linear.argtypes, lib.svdq_int4_linear.restype = [Shape, vp, vp, vp, vp, vp, vp, vp, vp], st
+    lib.svdq_deltaquant_sizes.argtypes = [i64, i64, i64, i64, P(sz), P(sz), P(sz)]
+    lib.svdq_deltaquant_sizes.restype = st
+    lib.svdq_deltaquant_encode.argtypes = [i64, i64, i64, i64, vp, vp, vp, vp, vp]
+    lib.svdq_deltaquant_encode.restype = st
     _lib = lib
     return lib
 
@@ -325,6 +329,30 @@ def svdq_int4_linear(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None,
     _check(load().svdq_int4_linear(shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t),
                                    _ptr(Y), _stream()))
     return Y
+
+
+# ---------------------------------------------------------------- DeltaQuant
+
+def svdq_deltaquant_sizes(F: int, H: int, W: int, C: int) -> tuple[int, int, int]:
+    a, b, c = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load().svdq_deltaquant_sizes(F, H, W, C, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return a.value, b.value, c.value
+
+
+def svdq_deltaquant_encode(X: torch.Tensor, dims: tuple[int, int, int], out: tuple | None = None):
+    """Core + delta encoding of video tokens X bf16 [F*H*W][C] (2 x 2 x 2 blocks).
+    Returns (core uint8 [blocks][C], delta codes uint8 [F*H*W][C/2], delta scales native uint8)."""
+    F, H, W = dims
+    C = X.shape[1]
+    if out is None:
+        cb, _, sb = svdq_deltaquant_sizes(F, H, W, C)
+        core = torch.empty(cb // C, C, dtype=torch.uint8, device=X.device)
+        Qd = torch.empty(F * H * W, C // 2, dtype=torch.uint8, device=X.device)
+        Sd = torch.empty(sb, dtype=torch.uint8, device=X.device)
+    else:
+        core, Qd, Sd = out
+    _check(load().svdq_deltaquant_encode(F, H, W, C, _ptr(X), _ptr(core), _ptr(Qd), _ptr(Sd), _stream()))
+    return core, Qd, Sd
 
 
 def svdq_selftest_timeout() -> None:
