@@ -186,37 +186,47 @@ SVDQ_API svdq_status svdq_linear(svdq_shape shape, const void* Qx, const void* S
                         const void* Sr, const void* L2t, void* Y, int variant, void* stream);
 
 /* svdq_linear whose output feeds another W4A4 layer directly: Y, quantized
- * for the NEXT layer (whose K equals this layer's N). Results are bit-identical
- * to the two calls
+ * for the NEXT layer (whose K equals this layer's N). The codes and scales are
+ * bit-identical to those of the two calls
  *     svdq_linear(shape, ..., Y);
  *     svdq_quantize_act({M, N, *, next_rank}, Y, next_inv_lambda, next_L1p,
  *                       next_Qx, next_Sx, next_T, SVDQ_FUSED, stream);
  * i.e. next_Qx codes [M][N/2], next_Sx native scales of Y's 16-groups along N
- * and, when next_rank > 0, next_T bf16 [M][next_rank] = bf16(Y next_L1p^T).
- * When next_rank == 0 and the shape runs on 256 x 256 CTA-pair tiles, the
- * GEMM's epilogue encodes the accumulator tile directly (walkthrough eq. (1)
- * and Fig. 6's activation quantization, moved into the producer of the
- * activation), so Y is written only if asked for; otherwise Y is formed (in
- * Y, or in the workspace when Y is NULL) and quantized by svdq_quantize_act's
- * kernel: the next layer's down-projection sums over all of N, and inside this
- * GEMM it would stall the tensor pipe (svdq_gemm_qnext.cuh).
+ * and, when next_rank > 0, next_T bf16 [M][next_rank] ~= Y next_L1p^T.
+ * Routes (walkthrough eq. (1) and Fig. 6's activation quantization, moved into
+ * the producer of the activation):
+ *   - next_rank == 0 and the shape runs on 256 x 256 CTA-pair tiles: the GEMM's
+ *     epilogue encodes the accumulator tile directly; Y is written only if
+ *     asked for.
+ *   - next_rank 16 or 32 on 256 x 256 pair tiles, with SVDQ_NEXT_FUSE_LOWRANK
+ *     in `flags`: the epilogue also forms the next layer's down-projection with
+ *     tcgen05 MMAs on the staged Y tile; each tile's fp32 partial of next_T
+ *     goes to the workspace and a second kernel adds them in tile order (next_T
+ *     then agrees with the two calls within bf16 rounding, not bit for bit).
+ *     Measured slower than the two calls on the FLUX projections, so it is
+ *     opt-in.
+ *   - otherwise Y is formed (in Y, or in the workspace when Y is NULL) and
+ *     quantized by svdq_quantize_act's kernel (next_T then bit-identical).
  * Inputs as for svdq_linear, plus next_inv_lambda fp32 [N] and next_L1p bf16
  * [next_rank][N] of the next layer (next_rank in {0, 16, ..., 128}; next_L1p and
  * next_T may be NULL when it is 0). Y bf16 [M][N] is written only if non-NULL.
- * workspace / workspace_bytes: when Y is NULL, at least
- * svdq_linear_quantize_next_workspace()'s size (0 on the fused path, M*N*2
- * otherwise); SVDQ_ERR_BUFFER_TOO_SMALL if smaller. Its contents on return are
+ * flags: 0 or SVDQ_NEXT_FUSE_LOWRANK; other bits are SVDQ_ERR_INVALID_ARG.
+ * workspace / workspace_bytes: at least svdq_linear_quantize_next_workspace()'s
+ * size for the same flags -- 0 on the rank-0 fused route, N/256*M*next_rank*4
+ * on the low-rank fused route, M*N*2 otherwise (needed there only when Y is
+ * NULL); SVDQ_ERR_BUFFER_TOO_SMALL if smaller. Its contents on return are
  * unspecified. Stream-ordered. */
+#define SVDQ_NEXT_FUSE_LOWRANK 1u
 SVDQ_API svdq_status svdq_linear_quantize_next(svdq_shape shape, const void* Qx, const void* Sx, const void* T,
                                                const void* Qr, const void* Sr, const void* L2t, int32_t next_rank,
                                                const float* next_inv_lambda, const void* next_L1p, void* next_Qx,
                                                void* next_Sx, void* next_T, void* Y, void* workspace,
-                                               size_t workspace_bytes, void* stream);
+                                               size_t workspace_bytes, unsigned int flags, void* stream);
 
-/* Workspace bytes svdq_linear_quantize_next needs for `shape` and next_rank on
- * the current device when it is given no Y (the kernel choice depends on the
- * device's SM count). */
-SVDQ_API svdq_status svdq_linear_quantize_next_workspace(svdq_shape shape, int32_t next_rank, size_t* bytes);
+/* Workspace bytes svdq_linear_quantize_next needs for `shape`, next_rank and
+ * flags on the current device (the route depends on the device's SM count). */
+SVDQ_API svdq_status svdq_linear_quantize_next_workspace(svdq_shape shape, int32_t next_rank, unsigned int flags,
+                                                         size_t* bytes);
 
 /* LoRA as part of the low-rank branch (walkthrough, Figure 9 and Figure 16: a
  * LoRA runs in, or is merged into, the independent 16-bit branch, with no

@@ -126,24 +126,26 @@ def test_linear_quantize_next_argument_checks(lib):
     bad = ctypes.c_void_p((1 << 20) + 8)
     sh = S.Shape(256, 512, 768, 16)
     ws = ctypes.c_size_t()
-    assert lib.svdq_linear_quantize_next_workspace(sh, 20, ctypes.byref(ws)) == 2       # next rank not a multiple of 16
-    assert lib.svdq_linear_quantize_next_workspace(sh, 144, ctypes.byref(ws)) == 2
-    assert lib.svdq_linear_quantize_next_workspace(sh, 32, None) == 1
-    assert lib.svdq_linear_quantize_next_workspace(S.Shape(0, 512, 768, 16), 32, ctypes.byref(ws)) == 0
+    assert lib.svdq_linear_quantize_next_workspace(sh, 20, 0, ctypes.byref(ws)) == 2    # next rank not a multiple of 16
+    assert lib.svdq_linear_quantize_next_workspace(sh, 144, 0, ctypes.byref(ws)) == 2
+    assert lib.svdq_linear_quantize_next_workspace(sh, 32, 0, None) == 1
+    assert lib.svdq_linear_quantize_next_workspace(sh, 32, 2, ctypes.byref(ws)) == 1   # unknown flag
+    assert lib.svdq_linear_quantize_next_workspace(S.Shape(0, 512, 768, 16), 32, 1, ctypes.byref(ws)) == 0
     assert ws.value == 0                                                                   # M == 0 needs none
     args = [good] * 6   # Qx, Sx, T, Qr, Sr, L2t
     nxt = [good] * 6    # next_inv_lambda, next_L1p, next_Qx, next_Sx, next_T, Y
-    assert lib.svdq_linear_quantize_next(sh, *args, 48, *nxt, good, 1 << 20, None) not in (0, 1, 3)  # device / shape only
-    assert lib.svdq_linear_quantize_next(sh, *args, 24, *nxt, good, 1 << 20, None) == 2
-    assert lib.svdq_linear_quantize_next(S.Shape(256, 512, 100, 16), *args, 16, *nxt, good, 1 << 20, None) == 2
-    assert lib.svdq_linear_quantize_next(sh, *args, 32, good, None, good, good, good, good, good, 1 << 20, None) == 1
-    assert lib.svdq_linear_quantize_next(sh, *args, 0, good, None, good, good, None, None, good, 1 << 20, None) != 1
-    assert lib.svdq_linear_quantize_next(sh, *args, 32, good, good, good, bad, good, good, good, 1 << 20, None) == 3
+    assert lib.svdq_linear_quantize_next(sh, *args, 48, *nxt, good, 1 << 20, 0, None) not in (0, 1, 3)  # device / shape only
+    assert lib.svdq_linear_quantize_next(sh, *args, 24, *nxt, good, 1 << 20, 0, None) == 2
+    assert lib.svdq_linear_quantize_next(sh, *args, 32, *nxt, good, 1 << 20, 4, None) == 1              # unknown flag
+    assert lib.svdq_linear_quantize_next(S.Shape(256, 512, 100, 16), *args, 16, *nxt, good, 1 << 20, 0, None) == 2
+    assert lib.svdq_linear_quantize_next(sh, *args, 32, good, None, good, good, good, good, good, 1 << 20, 0, None) == 1
+    assert lib.svdq_linear_quantize_next(sh, *args, 0, good, None, good, good, None, None, good, 1 << 20, 0, None) != 1
+    assert lib.svdq_linear_quantize_next(sh, *args, 32, good, good, good, bad, good, good, good, 1 << 20, 0, None) == 3
     assert lib.svdq_linear_quantize_next(S.Shape(0, 512, 768, 16), None, None, None, None, None, None, 32, None, None,
-                                         None, None, None, None, None, 0, None) == 0      # M == 0: a no-op
+                                         None, None, None, None, None, 0, 0, None) == 0   # M == 0: a no-op
     if not torch.cuda.is_available():
-        assert lib.svdq_linear_quantize_next(sh, *args, 32, *nxt, good, 1 << 20, None) == 5
-        assert lib.svdq_linear_quantize_next_workspace(sh, 32, ctypes.byref(ws)) == 5
+        assert lib.svdq_linear_quantize_next(sh, *args, 32, *nxt, good, 1 << 20, 0, None) == 5
+        assert lib.svdq_linear_quantize_next_workspace(sh, 32, 0, ctypes.byref(ws)) == 5
 
 
 def test_int4_sizes_and_argument_checks(lib):

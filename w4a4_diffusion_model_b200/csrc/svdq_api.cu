@@ -363,12 +363,12 @@ svdq_status launch_gemm_single(const svdq_shape& s, int rank, const void* Qx, co
 // Launch configuration of the pair kernel: clusters of 2 CTAs, and (for real
 // launches) programmatic stream serialization, so that the kernel's prologue
 // overlaps the end of the previous kernel of the stream. `attr` must hold 2.
-template <int NB>
+template <int NB, bool QLR = false>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribute* attr, bool pdl = true) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * clusters, 1, 1);
   cfg.blockDim = dim3(svdq::kGemmThreads, 1, 1);
-  cfg.dynamicSmemBytes = svdq::PairCfg<NB>::kBytes;
+  cfg.dynamicSmemBytes = svdq::PairCfg<NB, QLR>::kBytes;
   cfg.stream = st;
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -383,19 +383,19 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t st, cudaLaunchAttribut
 
 // Clusters of the pair kernel (tile width NB) that fit on the device at once,
 // cached per device; also sets the kernel's shared-memory attribute there.
-template <int NB, bool QNEXT = false>
+template <int NB, bool QNEXT = false, bool QLR = false>
 int pair_clusters() {
   static std::atomic<int> cache[kMaxDevices];
   // cached as count + 1; a failed attribute call is not cached
   return per_device_once(cache, current_device(), [] {
-    auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB>::kBytes) !=
+    auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT, QLR>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, svdq::PairCfg<NB, QLR>::kBytes) !=
         cudaSuccess) {
       cudaGetLastError();
       return 0;
     }
     cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = pair_config<NB>(sm_count() / 2, nullptr, attr, false);
+    cudaLaunchConfig_t cfg = pair_config<NB, QLR>(sm_count() / 2, nullptr, attr, false);
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, (void*)kern, &cfg) != cudaSuccess) {
       cudaGetLastError();
@@ -405,12 +405,14 @@ int pair_clusters() {
   }) - 1;
 }
 
-template <int NB, bool QNEXT = false>
+template <int NB, bool QNEXT = false, bool QLR = false>
 svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, const void* Sx, const void* T,
                              const void* Qr, const void* Sr, const void* L2t, void* Y, cudaStream_t st,
-                             int clusters, const svdq::NextQuant& nq = svdq::NextQuant{}, bool store_y = true) {
+                             int clusters, const svdq::NextQuant& nq = svdq::NextQuant{}, bool store_y = true,
+                             const void* next_L1p = nullptr) {
   constexpr uint32_t kBBox = NB == 256 ? 128 : 64;   // B rows per TMA box
-  CUtensorMap tqx, tqr, tsa, tsb, tt, tl, ty;
+  CUtensorMap tqx, tqr, tsa, tsb, tt, tl, ty, tl1n;
+  memset(&tl1n, 0, sizeof(tl1n));
   svdq_status r;
   if ((r = make_tmap(&tqx, Qx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)s.K / 2, (uint64_t)s.M, svdq::kGemmBKBytes,
                      128, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
@@ -438,13 +440,18 @@ svdq_status launch_gemm_pair(const svdq_shape& s, int rank, const void* Qx, cons
   } else {
     memset(&ty, 0, sizeof(ty));
   }
-  auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT>;
+  if (QLR) {   // the next layer's L1p' [next_rank][N]: boxes of 64 columns x next_rank/2 rows
+    if ((r = make_tmap(&tl1n, next_L1p, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)s.N, (uint64_t)nq.next_rank,
+                       64, (uint32_t)nq.next_rank / 2, CU_TENSOR_MAP_SWIZZLE_128B)) != SVDQ_OK)
+      return r;
+  }
+  auto kern = svdq::svdq_gemm_pair_kernel<NB, QNEXT, QLR>;
   const long long tiles = ((s.M + svdq::kPairBM - 1) / svdq::kPairBM) * (s.N / NB);
   const int ncl = (int)(tiles < clusters ? tiles : clusters);
   cudaLaunchAttribute attr[2];
-  cudaLaunchConfig_t cfg = pair_config<NB>(ncl, st, attr);
-  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, (int)s.M, (int)s.N, (int)s.K, rank, nq,
-                               store_y ? 1 : 0));
+  cudaLaunchConfig_t cfg = pair_config<NB, QLR>(ncl, st, attr);
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, kern, tqx, tqr, tsa, tsb, tt, tl, ty, tl1n, (int)s.M, (int)s.N, (int)s.K, rank,
+                               nq, store_y ? 1 : 0));
   SVDQ_LAUNCHED("svdq_gemm_pair_kernel");
   return SVDQ_OK;
 }
@@ -481,17 +488,24 @@ svdq_status launch_gemm(const svdq_shape& s, int rank, const void* Qx, const voi
   }
 }
 
-// The next layer's quantization runs in the GEMM epilogue when the next layer
-// has no low-rank branch and the shape takes the 256 x 256 pair kernel; every
-// other case forms Y (in the caller's Y or in the workspace) and runs the
-// quantizer on it. See svdq_gemm_qnext.cuh for why a low-rank next layer is
-// not fused.
-bool qnext_fused(const svdq_shape& s, int next_rank) {
-  return next_rank == 0 && gemm_choice(s) == 256 && pair_clusters<256, true>() > 0;
+// The next layer's quantization runs in the GEMM epilogue when the shape takes
+// the 256 x 256 pair kernel and the next layer's rank is 0, 16 or 32 (with a
+// low-rank branch the epilogue also forms the partial T' of each tile, summed
+// by tprime_reduce_kernel; svdq_gemm_qnext.cuh). Every other case forms Y (in
+// the caller's Y or in the workspace) and runs the quantizer on it.
+// The low-rank route is opt-in (SVDQ_NEXT_FUSE_LOWRANK): it measured slower
+// than the two-call route on the FLUX projections.
+bool qnext_fused(const svdq_shape& s, int next_rank, unsigned flags) {
+  if (gemm_choice(s) != 256) return false;
+  if (next_rank == 0) return pair_clusters<256, true>() > 0;
+  return (flags & SVDQ_NEXT_FUSE_LOWRANK) && (next_rank == 16 || next_rank == 32) &&
+         pair_clusters<256, true, true>() > 0;
 }
 
-size_t qnext_workspace_bytes(const svdq_shape& s, int next_rank) {
-  return qnext_fused(s, next_rank) ? 0 : (size_t)s.M * (size_t)s.N * 2u;
+size_t qnext_workspace_bytes(const svdq_shape& s, int next_rank, unsigned flags) {
+  if (!qnext_fused(s, next_rank, flags)) return (size_t)s.M * (size_t)s.N * 2u;
+  // fp32 partials of T' per 256-column tile: [N/256][M][next_rank]
+  return (size_t)(s.N / 256) * (size_t)s.M * (size_t)next_rank * 4u;
 }
 
 template <int RANK>
@@ -839,10 +853,11 @@ svdq_status svdq_linear(svdq_shape s, const void* Qx, const void* Sx, const void
   return launch_up_rmw(s, s.rank, T, L2t, Y, st);
 }
 
-svdq_status svdq_linear_quantize_next_workspace(svdq_shape s, int32_t next_rank, size_t* bytes) {
+svdq_status svdq_linear_quantize_next_workspace(svdq_shape s, int32_t next_rank, unsigned int flags, size_t* bytes) {
   g_last_error[0] = 0;
   svdq_status r = check_shape(s);
   if (r != SVDQ_OK) return r;
+  if (flags & ~SVDQ_NEXT_FUSE_LOWRANK) return fail(SVDQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   if (next_rank < 0 || next_rank > 128 || next_rank % 16)
     return fail(SVDQ_ERR_UNSUPPORTED_SHAPE, "next rank %d: need one of 0, 16, ..., 128", (int)next_rank);
   if (!bytes) return fail(SVDQ_ERR_INVALID_ARG, "null pointer");
@@ -851,7 +866,7 @@ svdq_status svdq_linear_quantize_next_workspace(svdq_shape s, int32_t next_rank,
     return SVDQ_OK;
   }
   if ((r = check_device()) != SVDQ_OK) return r;
-  *bytes = qnext_workspace_bytes(s, next_rank);
+  *bytes = qnext_workspace_bytes(s, next_rank, flags);
   return SVDQ_OK;
 }
 
@@ -859,10 +874,11 @@ svdq_status svdq_linear_quantize_next(svdq_shape s, const void* Qx, const void* 
                                       const void* Sr, const void* L2t, int32_t next_rank,
                                       const float* next_inv_lambda, const void* next_L1p, void* next_Qx,
                                       void* next_Sx, void* next_T, void* Y, void* workspace, size_t workspace_bytes,
-                                      void* stream) {
+                                      unsigned int flags, void* stream) {
   g_last_error[0] = 0;
   svdq_status r = check_shape(s);
   if (r != SVDQ_OK) return r;
+  if (flags & ~SVDQ_NEXT_FUSE_LOWRANK) return fail(SVDQ_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   const svdq_shape ns = {s.M, s.N, 128, next_rank};   // the next layer reads Y as its X (K' = N)
   if ((r = check_shape(ns)) != SVDQ_OK) return r;
   if (s.M == 0) return SVDQ_OK;
@@ -873,8 +889,8 @@ svdq_status svdq_linear_quantize_next(svdq_shape s, const void* Qx, const void* 
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return fail(SVDQ_ERR_MISALIGNED, "every pointer must be 16-byte aligned");
   if ((r = check_device()) != SVDQ_OK) return r;
-  const bool fused = qnext_fused(s, next_rank);
-  const size_t need = Y ? 0 : qnext_workspace_bytes(s, next_rank);
+  const bool fused = qnext_fused(s, next_rank, flags);
+  const size_t need = (Y && !fused) ? 0 : qnext_workspace_bytes(s, next_rank, flags);
   if (need > 0 && (workspace_bytes < need || !workspace))
     return fail(SVDQ_ERR_BUFFER_TOO_SMALL, "workspace of %zu bytes needed", need);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -887,8 +903,29 @@ svdq_status svdq_linear_quantize_next(svdq_shape s, const void* Qx, const void* 
   nq.inv_lambda = next_inv_lambda;
   nq.qx = static_cast<uint8_t*>(next_Qx);
   nq.sx = static_cast<uint8_t*>(next_Sx);
-  return launch_gemm_pair<256, true>(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<256, true>(), nq,
-                                     Y != nullptr);
+  nq.tp_ws = static_cast<float*>(workspace);
+  nq.next_rank = next_rank;
+  if (next_rank == 0)
+    return launch_gemm_pair<256, true>(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<256, true>(), nq,
+                                       Y != nullptr);
+  if ((r = launch_gemm_pair<256, true, true>(s, s.rank, Qx, Sx, T, Qr, Sr, L2t, Y, st, pair_clusters<256, true, true>(),
+                                             nq, Y != nullptr, next_L1p)) != SVDQ_OK)
+    return r;
+  // T' = the tiles' partials added in tile order, rounded to bf16
+  const long long n4 = s.M * (long long)next_rank / 4;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((unsigned)((n4 + 255) / 256), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  SVDQ_CUDA(cudaLaunchKernelEx(&cfg, svdq::tprime_reduce_kernel, static_cast<const float4*>(workspace),
+                               static_cast<__nv_bfloat16*>(next_T), n4, (int)(s.N / 256)));
+  SVDQ_LAUNCHED("tprime_reduce_kernel");
+  return SVDQ_OK;
 }
 
 namespace svdq {

@@ -28,6 +28,8 @@ constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kSfWarp0 = 10;
 constexpr int kSfWarps = 4;
+// 14 warps: one SM sub-partition (16384 registers) holds 4 of them, so a
+// thread may use at most 128 registers.
 constexpr int kGemmThreads = 32 * (kGemmEpiWarps + 2 + kSfWarps);
 
 // TMEM: accumulator columns [0, 256); then one scale buffer of 48 columns per

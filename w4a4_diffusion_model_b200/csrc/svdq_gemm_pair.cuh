@@ -44,21 +44,31 @@ constexpr int kPairBM = 256;                          // M rows per pair tile (1
 constexpr int kPairStageA = 128 * kGemmBKBytes;       // 16 KB: this CTA's 128 Qx rows (or T rows)
 constexpr int kPairStageSfa = kGemmKBPerStage * kSfAtomBytes;       // 2 KB
 
-template <int NB>
+// QLR: the epilogue also forms the next layer's down-projection (next rank 16
+// or 32): a ring of 4 stages (so that TMEM keeps 32 columns for T' and shared
+// memory two staging boxes per epilogue warp and the tile's L1p' slice).
+template <int NB, bool QLR = false>
 struct PairCfg {
   static_assert(NB == 256 || NB == 384, "pair tile width");
+  static_assert(!QLR || NB == 256, "the next layer's down-projection runs on 256 x 256 tiles");
   static constexpr int kBRows = NB / 2;                               // B rows per CTA
   static constexpr int kStageB = kBRows * kGemmBKBytes;               // 16 | 24 KB
   static constexpr int kSfbBlocks = NB / 128;                         // 128-row blocks of B scales
   static constexpr int kStageSfb = kSfbBlocks * kGemmKBPerStage * kSfAtomBytes;   // 4 | 6 KB
   static constexpr int kStageBytes = kPairStageA + kStageB + kPairStageSfa + kStageSfb;   // 38 | 48 KB
-  static constexpr int kStages = NB == 256 ? 5 : 4;
+  static constexpr int kStages = QLR ? 4 : NB == 256 ? 5 : 4;
   static constexpr uint32_t kSfCols = 4 * kGemmKBPerStage * (1 + kSfbBlocks);   // 48 | 64 TMEM columns
-  static constexpr int kSfBufs = (int)((kTmemCols - NB) / kSfCols);             // 5 | 2
+  static constexpr uint32_t kTpCols = QLR ? 32 : 0;                             // T' accumulator columns
+  static constexpr int kSfBufs = (int)((kTmemCols - NB - kTpCols) / kSfCols);   // 5 | 2 (4 with QLR)
+  static constexpr uint32_t kTpCol = kTmemCols - kTpCols;                       // T' at columns [480, 512)
   static constexpr bool kSfPerStage = kSfBufs >= kStages;
   static_assert(kSfBufs >= 2, "scale buffers");
+  static_assert(NB + kSfBufs * kSfCols <= kTpCol, "TMEM plan");
+  static constexpr int kEpiBoxes = QLR ? 2 : 1;                                 // staging boxes per epilogue warp
   static constexpr int kEpiOffset = kStages * kStageBytes;
-  static constexpr int kBarOffset = kEpiOffset + kGemmEpiWarps * kEpiBoxBytes;
+  static constexpr int kL1Half = 2 * 16 * 128;   // L1p' columns of one tile half: 2 boxes of <= 16 rows x 64
+  static constexpr int kL1Offset = kEpiOffset + kGemmEpiWarps * kEpiBoxes * kEpiBoxBytes;
+  static constexpr int kBarOffset = kL1Offset + (QLR ? 2 * kL1Half : 0);
   static constexpr int kBytes = kBarOffset + 512 + 1024;
   // TMEM column of the scale buffer of item `it` in ring stage `s`
   __device__ static uint32_t sf_col(uint32_t it, int s) {
@@ -66,20 +76,176 @@ struct PairCfg {
   }
 };
 
+// Epilogue of one warp (q = lane quadrant, h = column half) when the next
+// layer has a low-rank branch. Per tile:
+//   1. drain the accumulator (bf16-packed) and release it to the MMA issuer;
+//   2. write the next layer's codes and scales (epilogue_encode_next);
+//   3. stage the band's two 64-column boxes b (rows of this CTA, bf16 Y) in
+//      the warp's own boxes -- the four warps of a half form one 128 x 64
+//      K-major operand per b -- store them to Y if asked, and report each to
+//      the even CTA (ych_full[h][b]). One thread (even CTA, warp q = 0, h = 1)
+//      issues the T' MMAs of every chunk in the order (b, h) = (0,0), (0,1),
+//      (1,0), (1,1): D (TMEM columns kTpCol.., both CTAs) += Y chunk x L1p'
+//      chunk^T, committing each chunk to ych_empty[h][b] and the tile to
+//      tp_full;
+//   4. the warps of half 0 read T' (their 32 lanes) and write the tile's fp32
+//      partial to nq.tp_ws[tile column][row][:], then report tp_empty.
+// Warps q = 0 of each CTA TMA-load the L1p' columns of their half (the B rows
+// of this CTA: next_rank/2 of them) for each tile into l1_full[h], after the
+// previous tile's T' MMAs have completed. Each barrier completes once per
+// tile, so parity waits cannot alias across tiles.
+template <class C>
+__device__ __forceinline__ void epilogue_next_lowrank(
+    unsigned char* smem, uint32_t tmem, uint32_t crank, bool leader, int q, int h, int lane, int cluster,
+    int nclusters, int ntiles, int tiles_n, int M, int N, const NextQuant& nq, const float2* rcp_tbl,
+    const void* tm_y, const void* tm_l1n, bool store_y, uint64_t* acc_full, uint64_t* acc_empty,
+    uint64_t* ych_full, uint64_t* ych_empty, uint64_t* tp_full, uint64_t* tp_empty, uint64_t* l1_full,
+    uint64_t* tp_drain) {
+  const int rh = nq.next_rank / 2;                              // L1p' rows per CTA (B rows of the pair MMA)
+  const uint32_t l1_bytes = 2u * (uint32_t)rh * 128u;
+  unsigned char* l1buf = smem + C::kL1Offset + h * C::kL1Half;
+  const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
+  const uint32_t tp_empty_leader = mapa_shared(smem_u32(tp_empty), 0);
+  const bool loader = q == 0 && lane == 0;
+  const bool issuer = leader && q == 0 && h == 1 && lane == 0;
+  const uint32_t idesc_tp = idesc_bf16(kPairBM, nq.next_rank);
+  uint32_t l1_issued = 0;
+  auto load_l1 = [&](int tile) {
+    const int n0 = (tile % tiles_n) * 256 + h * 128;
+    ++l1_issued;
+    mbar_arrive_expect_tx(l1_full + h, l1_bytes);
+    tma_load_2d(l1buf, tm_l1n, l1_full + h, n0, (int)crank * rh);
+    tma_load_2d(l1buf + rh * 128, tm_l1n, l1_full + h, n0 + 64, (int)crank * rh);
+  };
+  if (loader && cluster < ntiles) load_l1(cluster);
+  bool ok = true;
+  uint32_t tcount = 0;
+  for (int tile = cluster; tile < ntiles && ok; tile += nclusters, ++tcount) {
+    const int m0 = (tile / tiles_n) * kPairBM + 128 * (int)crank;
+    const int n0 = (tile % tiles_n) * 256;
+    const uint32_t par = tcount & 1u;
+    const float4 inv4 = epilogue_inv_factors(nq, n0 + h * 128, lane);
+    ok = mbar_wait(acc_full, par, kDevErrTimeoutAccum) && !device_error_set();
+    ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;   // one decision per warp
+    tc_fence_after();
+    if (!ok) break;
+    const uint32_t taddr = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 128);
+    uint32_t p[64];
+    epilogue_drain_pack<4>(taddr, p);
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+    epilogue_encode_next<2>(p, nq, rcp_tbl, inv4, m0 + 32 * q, n0 + h * 128, M, N, lane);
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      unsigned char* box = smem + C::kEpiOffset + ((h * 2 + b) * 4 + q) * kEpiBoxBytes;
+      if (lane == 0) {
+        // the box's previous T' MMAs and its previous Y store have read it
+        if (tcount > 0 && !mbar_wait(ych_empty + h * 2 + b, par ^ 1u, kDevErrTimeoutNext)) ok = false;
+        bulk_wait_read<1>();
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      epilogue_stage_box(&p[32 * b], box, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        if (q == 0 && b == 0 && !mbar_wait(l1_full + h, par, kDevErrTimeoutNext)) ok = false;
+        if (ok) mbar_arrive_remote(mapa_shared(smem_u32(ych_full + h * 2 + b), 0));
+        if (store_y && m0 + 32 * q < M) {
+          tma_store_2d_evict_first(tm_y, box, n0 + h * 128 + 64 * b, m0 + 32 * q);
+        }
+        bulk_commit();   // one group per box, stored or not, so that bulk_wait_read<1> keeps its meaning
+      }
+      if (issuer && ok) {
+#pragma unroll 1
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+          if (!mbar_wait(ych_full + hh * 2 + b, par, kDevErrTimeoutNext)) {
+            ok = false;
+            break;
+          }
+          if (b == 0 && hh == 0 && tcount > 0 && !mbar_wait(tp_empty, par ^ 1u, kDevErrTimeoutNext)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = smem_desc(smem_u32(smem + C::kEpiOffset + (hh * 2 + b) * 4 * kEpiBoxBytes), 16, 1024,
+                                        kSwizzle128B);
+          const uint64_t bd = smem_desc(smem_u32(smem + C::kL1Offset + hh * C::kL1Half + b * rh * 128), 16, 1024,
+                                        kSwizzle128B);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)   // 16 bf16 (32 bytes) of the chunk's 64 columns per MMA
+            mma_bf16_pair(tmem + C::kTpCol, ad + 2u * j, bd + 2u * j, idesc_tp, (b | hh | j) != 0 ? 1u : 0u);
+          tc_commit_pair(ych_empty + hh * 2 + b, 0x3);
+        }
+        if (ok && b == 1) tc_commit_pair(tp_full, 0x3);
+      }
+      __syncwarp();
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+    }
+    if (!ok) break;
+    // the tile's T' partial
+    if (h == 0) {
+      ok = mbar_wait(tp_full, par, kDevErrTimeoutNext);
+      ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
+      tc_fence_after();
+      if (!ok) break;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + ((uint32_t)(q * 32) << 16) + C::kTpCol, v);
+      tmem_ld_wait();
+      const int row = m0 + 32 * q + lane;
+      if (row < M) {
+        float4* dst = reinterpret_cast<float4*>(nq.tp_ws + ((size_t)(tile % tiles_n) * (size_t)M + (size_t)row) *
+                                                               (size_t)nq.next_rank);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (4 * i < nq.next_rank)
+            dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                 __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(tp_empty_leader);
+    }
+    // the next tile's L1p' columns, once this tile's T' MMAs are done with the buffer
+    if (q == 0) {
+      bool lok = true;
+      if (lane == 0 && tile + nclusters < ntiles) {
+        if (h == 1) lok = mbar_wait(tp_full, par, kDevErrTimeoutNext);
+        if (lok) load_l1(tile + nclusters);
+      }
+      ok = __shfl_sync(0xFFFFFFFFu, lok ? 1 : 0, 0) != 0;
+    }
+  }
+  // leave no TMA load of L1p' in flight (the last one was consumed already
+  // unless the loop stopped early; waiting on a completed phase returns at once)
+  if (loader && l1_issued > 0) mbar_wait(l1_full + h, (l1_issued - 1u) & 1u, kDevErrTimeoutNext);
+  // and no T' MMA running when TMEM is freed
+  if (issuer && tcount + (ok ? 0u : 1u) > 0) {
+    tc_commit_pair(tp_drain, 0x1);
+    mbar_wait(tp_drain, 0, kDevErrTimeoutNext);
+  }
+}
+
 // Launched with a cluster dimension of (2, 1, 1).
 // tm_qr / tm_l2 boxes are 128 rows (NB = 256) or 64 rows (NB = 384).
 // tm_sfa / tm_sfb view a native scale buffer as 3-D uint8
 // [row blocks][K/64 * 2 chunks][256 bytes]; box {256, 8, 1 | NB/128} (4 atoms per row block).
 // QNEXT: the epilogue also quantizes Y for the next layer (svdq_gemm_qnext.cuh),
 // and stores Y itself only when store_y is set.
-template <int NB, bool QNEXT = false>
+// QLR (with QNEXT): the next layer has a low-rank branch; tm_l1n views its
+// L1p' [next_rank][N] bf16 with boxes of 64 columns x next_rank/2 rows.
+template <int NB, bool QNEXT = false, bool QLR = false>
 __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     const __grid_constant__ CUtensorMap tm_qx, const __grid_constant__ CUtensorMap tm_qr,
     const __grid_constant__ CUtensorMap tm_sfa, const __grid_constant__ CUtensorMap tm_sfb,
     const __grid_constant__ CUtensorMap tm_t, const __grid_constant__ CUtensorMap tm_l2,
-    const __grid_constant__ CUtensorMap tm_y, int M, int N, int K, int rank, NextQuant nq, int store_y) {
+    const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_l1n, int M, int N, int K,
+    int rank, NextQuant nq, int store_y) {
   static_assert(!QNEXT || NB == 256, "the next layer's quantization runs on 256 x 256 tiles");
-  using C = PairCfg<NB>;
+  static_assert(!QLR || QNEXT, "the next layer's down-projection comes with its quantization");
+  using C = PairCfg<NB, QLR>;
   constexpr int STAGES = C::kStages;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -89,7 +255,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
   uint64_t* acc_full = sf_ready + STAGES;
   uint64_t* acc_empty = acc_full + 1;       // even CTA: both CTAs' epilogue warps report here
   uint64_t* mma_drain = acc_empty + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_drain + 1);
+  // QLR only: chunk (h, b) of the staged Y is in both CTAs (even CTA, 8 warp
+  // arrivals) / has been read by its T' MMAs (both CTAs, commit); the tile's
+  // T' partial is complete (both CTAs, commit) / has been read out (even CTA,
+  // 8 warp arrivals); this CTA's L1p' half h has landed
+  uint64_t* ych_full = mma_drain + 1;       // [h * 2 + b]
+  uint64_t* ych_empty = ych_full + 4;       // [h * 2 + b]
+  uint64_t* tp_full = ych_empty + 4;
+  uint64_t* tp_empty = tp_full + 1;
+  uint64_t* l1_full = tp_empty + 1;         // [h]
+  uint64_t* tp_drain = l1_full + 2;         // the T' issuer's MMAs have all completed (before TMEM is freed)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tp_drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t crank = cluster_ctarank();
@@ -110,6 +286,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, 2 * kGemmEpiWarps);
     mbar_init(mma_drain, 1);
+    if (QLR) {
+      for (int i = 0; i < 4; ++i) {
+        mbar_init(ych_full + i, 2 * 4);
+        mbar_init(ych_empty + i, 1);
+      }
+      mbar_init(tp_full, 1);
+      mbar_init(tp_empty, 2 * 4);
+      mbar_init(l1_full, 1);
+      mbar_init(l1_full + 1, 1);
+      mbar_init(tp_drain, 1);
+    }
     fence_mbar_init();
   }
   __shared__ float2 rcp_tbl[QNEXT ? 128 : 1];   // bracket of 1/s per E4M3 byte with the sign bit clear
@@ -127,6 +314,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       prefetch_tmap(&tm_t);
       prefetch_tmap(&tm_l2);
     }
+    if (QLR) prefetch_tmap(&tm_l1n);
   }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised, TMEM allocated in both
@@ -316,10 +504,16 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
     unsigned char* box = smem + C::kEpiOffset + warp * kEpiBoxBytes;
     const uint32_t acc_empty_leader = mapa_shared(smem_u32(acc_empty), 0);
     if (lane == 0 && (!QNEXT || store_y)) prefetch_tmap(&tm_y);
+    if constexpr (QLR) {
+      epilogue_next_lowrank<C>(smem, tmem, crank, leader, q, h, lane, cluster, nclusters, ntiles, tiles_n, M, N, nq,
+                               rcp_tbl, &tm_y, &tm_l1n, store_y != 0, acc_full, acc_empty, ych_full, ych_empty,
+                               tp_full, tp_empty, l1_full, tp_drain);
+    } else {
     uint32_t tcount = 0;
     for (int tile = cluster; tile < ntiles; tile += nclusters, ++tcount) {
       const int m0 = (tile / tiles_n) * kPairBM + 128 * (int)crank;
       const int n0 = (tile % tiles_n) * NB;
+      const float4 inv4 = QNEXT ? epilogue_inv_factors(nq, n0 + h * 128, lane) : make_float4(0.f, 0.f, 0.f, 0.f);
       const bool ok = mbar_wait(acc_full, tcount & 1u, kDevErrTimeoutAccum);
       tc_fence_after();
       if (!ok || device_error_set()) break;
@@ -333,7 +527,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         __syncwarp();
         if (lane == 0) mbar_arrive_remote(acc_empty_leader);   // this warp's part of the accumulator is drained
         if (QNEXT)
-          epilogue_quantize_next<2>(p, box, nq, rcp_tbl, &tm_y, store_y != 0, m0 + 32 * q, n0 + h * 128, M, N, lane);
+          epilogue_quantize_next<2>(p, box, nq, rcp_tbl, inv4, &tm_y, store_y != 0, m0 + 32 * q, n0 + h * 128, M, N,
+                                    lane);
         else
           epilogue_store_band<2>(p, box, &tm_y, n0 + h * 128, m0 + 32 * q, lane, store);
       } else {   // drain all 192 columns before releasing the accumulator, then store
@@ -345,6 +540,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
         epilogue_store_band<2>(p, box, &tm_y, n0 + h * 192, m0 + 32 * q, lane, store);
         epilogue_store_band<1>(p2, box, &tm_y, n0 + h * 192 + 128, m0 + 32 * q, lane, store);
       }
+    }
     }
     if (lane == 0) bulk_wait<0>();
   }

@@ -13,13 +13,15 @@
 // codes and the scale bytes in the native tile layout, and stores its band of
 // Y (TMA, as the plain epilogue does) only when the caller asked for Y.
 //
-// The next layer's low-rank down-projection T' = Y L1p'^T is not formed here:
-// it sums over all N, i.e. over every tile of a row, and on this kernel it
-// would have to run either as warp-level MMAs, which wait for the tcgen05 MMAs
-// of the running mainloop (measured: +46 us on the FLUX MLP-up projection for
-// a rank of 16), or as tcgen05 MMAs, for whose operands the 256 x 256 pair
-// tiles leave no shared or tensor memory. A next layer with a low-rank branch
-// therefore goes through Y and the quantizer (svdq_api.cu).
+// With a next layer that has a low-rank branch (rank 16 or 32), the epilogue
+// also forms that layer's down-projection T' = Y L1p'^T, which sums over all N
+// columns, i.e. over every tile of a row: each tile's bf16 Y, staged in
+// 128B-swizzled shared-memory boxes, is the A operand of tcgen05 bf16 pair
+// MMAs against the tile's 256 columns of L1p' (TMA-loaded per tile), into a
+// 32-column TMEM region; one epilogue thread of the even CTA issues them in a
+// fixed order. The tile's fp32 partial of T' goes to the caller's workspace
+// [N/256][M][rank'], and tprime_reduce_kernel adds the partials in tile order
+// and rounds T' to bf16 (svdq_gemm_pair.cuh, svdq_api.cu).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -36,14 +38,26 @@ struct NextQuant {
   const float* inv_lambda;        // [N] fp32 1/lambda' of the next layer
   uint8_t* qx;                    // [M][N/2] packed E2M1 codes
   uint8_t* sx;                    // native E4M3 scales of [ceil(M/128)*128][N/16]
+  float* tp_ws;                   // [N/256][M][next_rank] fp32 partials of T' (next_rank > 0)
+  int next_rank;                  // 0, 16 or 32
 };
 
-// Epilogue of one warp: quantize its band for the next layer, then store the
-// band of Y if asked (through the warp's 128B-swizzled staging box).
+// The warp's inverse smoothing factors for columns col0 + [0, 128): lane l
+// holds col0 + 4l .. 4l + 3. Loaded before the accumulator wait, so that the
+// load's latency hides behind it; the encoder fetches a group's 16 factors
+// from the four lanes that hold them.
+__device__ __forceinline__ float4 epilogue_inv_factors(const NextQuant& nq, int col0, int lane) {
+  return __ldg(reinterpret_cast<const float4*>(nq.inv_lambda + col0) + lane);
+}
+
+// One warp's band, quantized for the next layer from the packed bf16
+// registers: packed codes and native scale words (32 rows x 64*BOXES columns,
+// BOXES <= 2; inv4 from epilogue_inv_factors at col0).
 template <int BOXES>
-__device__ __forceinline__ void epilogue_quantize_next(const uint32_t (&p)[32 * BOXES], unsigned char* box,
-                                                       const NextQuant& nq, const float2* rcp_tbl, const void* tm_y,
-                                                       bool store_y, int row0, int col0, int M, int N, int lane) {
+__device__ __forceinline__ void epilogue_encode_next(const uint32_t (&p)[32 * BOXES], const NextQuant& nq,
+                                                     const float2* rcp_tbl, float4 inv4, int row0, int col0, int M,
+                                                     int N, int lane) {
+  static_assert(BOXES <= 2, "32 lanes x 4 factors cover 128 columns");
   const int row = row0 + lane;
   const int mpad = (M + 127) & ~127;
 #pragma unroll
@@ -52,16 +66,66 @@ __device__ __forceinline__ void epilogue_quantize_next(const uint32_t (&p)[32 * 
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int g = 4 * q + j;
+      float4 l[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k)   // factors 16g + 4k .. 16g + 4k + 3 sit in lane 4g + k
+        l[k] = make_float4(__shfl_sync(0xFFFFFFFFu, inv4.x, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.y, 4 * g + k),
+                           __shfl_sync(0xFFFFFFFFu, inv4.z, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.w, 4 * g + k));
       uint2 codes;
       uint32_t sb;
-      encode_group_bf16(&p[8 * g], nq.inv_lambda + col0 + 16 * g, rcp_tbl, codes, sb);
+      encode_group_vals(&p[8 * g], l, rcp_tbl, codes, sb);
       if (row < M) *reinterpret_cast<uint2*>(nq.qx + (size_t)row * (size_t)(N >> 1) + ((col0 + 16 * g) >> 1)) = codes;
       word |= sb << (8 * j);
     }
     // rows past M carry zero accumulators, hence the zero scales of the padding rows
     if (row < mpad) *reinterpret_cast<uint32_t*>(nq.sx + native_scale_offset(row, (col0 >> 4) + 4 * q, N)) = word;
   }
+}
+
+// Epilogue of one warp: quantize its band for the next layer, then store the
+// band of Y if asked (through the warp's 128B-swizzled staging box).
+template <int BOXES>
+__device__ __forceinline__ void epilogue_quantize_next(const uint32_t (&p)[32 * BOXES], unsigned char* box,
+                                                       const NextQuant& nq, const float2* rcp_tbl, float4 inv4,
+                                                       const void* tm_y, bool store_y, int row0, int col0, int M,
+                                                       int N, int lane) {
+  epilogue_encode_next<BOXES>(p, nq, rcp_tbl, inv4, row0, col0, M, N, lane);
   if (store_y) epilogue_store_band<BOXES>(p, box, tm_y, col0, row0, lane, row0 < M);
+}
+
+// Write box b (64 columns) of a warp's band into its 128B-swizzled staging
+// box: row `lane`, 16-byte chunk c at (c ^ (lane & 7)).
+__device__ __forceinline__ void epilogue_stage_box(const uint32_t* p, unsigned char* box, int lane) {
+  const uint32_t box_addr = smem_u32(box);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const uint32_t addr = box_addr + lane * 128 + ((c ^ (lane & 7)) << 4);
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(p[4 * c]), "r"(p[4 * c + 1]),
+                 "r"(p[4 * c + 2]), "r"(p[4 * c + 3])
+                 : "memory");
+  }
+}
+
+// T' = sum over the N/256 column tiles of their fp32 partials, in tile order,
+// rounded to bf16: ws [slices][M][r], T [M][r]. Four outputs per thread.
+__global__ void __launch_bounds__(256) tprime_reduce_kernel(const float4* __restrict__ ws,
+                                                            __nv_bfloat16* __restrict__ T, long long n4,
+                                                            int slices) {
+  grid_dependency_wait();     // the GEMM that wrote the partials is complete
+  grid_launch_dependents();
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n4) return;
+  float4 s = ws[i];
+  for (int t = 1; t < slices; ++t) {
+    const float4 v = ws[(long long)t * n4 + i];
+    s.x = __fadd_rn(s.x, v.x);
+    s.y = __fadd_rn(s.y, v.y);
+    s.z = __fadd_rn(s.z, v.z);
+    s.w = __fadd_rn(s.w, v.w);
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(s.x, s.y), hi = __floats2bfloat162_rn(s.z, s.w);
+  reinterpret_cast<uint2*>(T)[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&lo),
+                                              *reinterpret_cast<const uint32_t*>(&hi));
 }
 
 }  // namespace svdq

@@ -21,6 +21,7 @@ enum DeviceError : unsigned int {
   kDevErrTimeoutTmem = 4,     // waited too long for a TMEM allocation/free slot
   kDevErrTimeoutScales = 5,   // waited too long for a TMEM scale buffer (ready or free)
   kDevErrSelfTest = 6,        // the diagnostic wait of svdq_selftest_timeout gave up (as it must)
+  kDevErrTimeoutNext = 7,     // the next-layer down-projection in the GEMM epilogue waited too long
 };
 
 // Bound on any spin-wait inside a kernel, in nanoseconds of %globaltimer.

@@ -37,28 +37,27 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 // every fp32 v. Rounding is monotone, so when both products give the same
 // code that code is the exact one. They differ only when a midpoint lies in
 // the bracket (relative width < 2^-19.9, so at most one midpoint, and the two
-// codes are neighbours); then |v| is compared with that midpoint times s,
-// which is exact in fp32 (midpoints carry at most 4 significant bits, scales
-// at most 11), and a tie goes to the even code.
+// codes are neighbours); then |v| is compared with the midpoint above the
+// lower code, times s, which is exact in fp32 (midpoints carry at most 4
+// significant bits, scales at most 11), and a tie goes to the even code.
 __device__ __forceinline__ float2 recip_bracket(float s) {
   const float r = __frcp_rn(s);
   return make_float2(__fmul_rn(r, 1.0f - 0x1p-21f), __fmul_rn(r, 1.0f + 0x1p-21f));
 }
 
-// Value of the E2M1 magnitude code c (0..7): 0, 0.5, 1, 1.5, 2, 3, 4, 6.
-__device__ __forceinline__ float e2m1_value(uint32_t c) {
-  return c >= 2u ? __uint_as_float((((c >> 1) + 126u) << 23) | ((c & 1u) << 22)) : 0.5f * (float)c;
-}
-
-// The exact code of v / s given the codes a (of v lo) and b (of v hi) of its
-// bracket; the sign bit is the products' (kept for values rounding to zero).
-__device__ __forceinline__ uint32_t e2m1_resolve(float v, float s, uint32_t a, uint32_t b) {
-  if (a == b) return a;
-  const uint32_t m = a & 7u;                                            // b & 7 == m + 1
-  const float t = __fmul_rn(0.5f * (e2m1_value(m) + e2m1_value(m + 1u)), s);   // exact
+// The exact code of v / s, given the code a of the lower bracket product
+// v lo (sign bit included; the code of v hi is a or its upper neighbour):
+// compare |v| with the midpoint above a's magnitude m, times s (exact in fp32:
+// 4 x midpoint, looked up as a byte -- 1, 3, 5, 7, 10, 14, 20 for m = 0..6,
+// 255 for m = 7, where nothing lies above -- times s / 4). Above it: m + 1;
+// on it: the even one of m, m + 1; below it: m. Branch-free, so that a warp
+// whose lanes need it for different elements runs it once.
+__device__ __forceinline__ uint32_t e2m1_exact_nibble(float v, float s4, uint32_t a) {
+  const uint32_t m = a & 7u;
+  const float t = __fmul_rn((float)(__byte_perm(0x07050301u, 0xFF140E0Au, m) & 0xFFu), s4);   // exact
   const float x = fabsf(v);
-  const uint32_t mag = x > t ? m + 1u : x < t ? m : (m + (m & 1u));
-  return mag | (b & 8u);
+  const uint32_t up = (x > t || (x == t && (m & 1u))) ? 1u : 0u;
+  return (m + up) | (a & 8u);
 }
 
 // E2M1 byte (element 2i low, 2i+1 high) of a pair scaled by `inv`.
@@ -67,20 +66,19 @@ __device__ __forceinline__ uint32_t e2m1_pair(float2 v, float inv) {
                                             cudaRoundNearest) & 0xFFu;
 }
 
-// Packed codes of 8 pairs (16 values, one NVFP4 group) given the bracket of
-// 1/s: two 32-bit words, pair i in byte i % 4 of word i / 4. `lo`/`hi` are the
-// codes of the two products; the rare differing nibbles are resolved exactly.
+// Packed codes of 8 pairs (16 values, one NVFP4 group) given the codes of the
+// two bracket products (`lo`, `hi`; pair i in byte i % 4 of word i / 4): when
+// they differ anywhere, every element is recomputed exactly from `lo` (for an
+// element whose bracket holds no midpoint the recomputation returns its code).
 __device__ __forceinline__ uint2 e2m1_group_exact(const float2 (&v)[8], float s, uint2 lo, uint2 hi) {
   if (((lo.x ^ hi.x) | (lo.y ^ hi.y)) == 0u) return lo;
-  uint32_t w[2] = {lo.x, lo.y};
-  const uint32_t h[2] = {hi.x, hi.y};
+  const float s4 = 0.25f * s;
+  uint32_t w[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int sh = 8 * (i & 3);
-    const uint32_t a = (w[i >> 2] >> sh) & 0xFFu, b = (h[i >> 2] >> sh) & 0xFFu;
-    if (a == b) continue;
-    const uint32_t byte = e2m1_resolve(v[i].x, s, a & 15u, b & 15u) | (e2m1_resolve(v[i].y, s, a >> 4, b >> 4) << 4);
-    w[i >> 2] = (w[i >> 2] & ~(0xFFu << sh)) | (byte << sh);
+    const uint32_t a = ((i < 4 ? lo.x : lo.y) >> (8 * (i & 3))) & 0xFFu;
+    const uint32_t byte = e2m1_exact_nibble(v[i].x, s4, a & 15u) | (e2m1_exact_nibble(v[i].y, s4, a >> 4) << 4);
+    w[i >> 2] |= byte << (8 * (i & 3));
   }
   return make_uint2(w[0], w[1]);
 }

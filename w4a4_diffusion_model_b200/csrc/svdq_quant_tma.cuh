@@ -106,19 +106,18 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
 }
 
 // The NVFP4 recipe of nvfp4_encode16 for one group given as 8 packed bf16
-// pairs and its 16 inverse smoothing factors:
+// pairs and its 16 inverse smoothing factors (l[q] holds factors 4q..4q+3):
 //   v = fp32(x * inv_lambda); s = E4M3_rne_satfinite(fp32(max|v| / 6));
 //   q = E2M1_rne_satfinite(v / s) of the exact quotient, all +0 when s is 0.
 // The bracket (lo, hi) of 1/s comes from `rcp_tbl`, indexed by the E4M3 byte
 // of s (recip_bracket of its value).
-__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float2* rcp_tbl,
+__device__ __forceinline__ void encode_group_vals(const uint32_t* w, const float4 (&l)[4], const float2* rcp_tbl,
                                                   uint2& codes, uint32_t& sbyte) {
   float2 v[8];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const float4 l = *reinterpret_cast<const float4*>(il + 4 * q);
-    v[2 * q] = mul2_rn(make_float2(bf16lo(w[2 * q]), bf16hi(w[2 * q])), make_float2(l.x, l.y));
-    v[2 * q + 1] = mul2_rn(make_float2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1])), make_float2(l.z, l.w));
+    v[2 * q] = mul2_rn(make_float2(bf16lo(w[2 * q]), bf16hi(w[2 * q])), make_float2(l[q].x, l[q].y));
+    v[2 * q + 1] = mul2_rn(make_float2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1])), make_float2(l[q].z, l[q].w));
   }
   float m[8];
 #pragma unroll
@@ -151,6 +150,15 @@ __device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float
   codes = e2m1_group_exact(v, sval, make_uint2(lo[0], lo[1]), make_uint2(hi[0], hi[1]));
 }
 
+// The same with the 16 inverse smoothing factors read from `il` (any space).
+__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float2* rcp_tbl,
+                                                  uint2& codes, uint32_t& sbyte) {
+  float4 l[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) l[q] = *reinterpret_cast<const float4*>(il + 4 * q);
+  encode_group_vals(w, l, rcp_tbl, codes, sbyte);
+}
+
 // Bracketing reciprocals of every E4M3 scale byte with the sign bit clear
 // (byte 0, a zero scale, is never looked up).
 __device__ __forceinline__ float2 e4m3_recip_bracket(uint32_t byte) {
@@ -178,7 +186,6 @@ enum QuantCodec : int {
 // FP8 tensor-core MMA reads; the scale is returned as its fp32 value.
 // Every lane of the warp must call it (quad shuffles).
 __device__ __forceinline__ float int4_resolve(float v, float s, float qa, float qb) {
-  if (qa == qb) return qa;
   const float m = fminf(fabsf(qa), fabsf(qb));
   const float t = __fmul_rn(m + 0.5f, s);   // exact
   const float x = fabsf(v);

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libsvdq.so")
 SVDQ_FUSED = 0
 SVDQ_UNFUSED = 1
 SVDQ_PREPARE_GIVEN_FACTORS = 1
+SVDQ_NEXT_FUSE_LOWRANK = 1
 
 STATUS = {
     0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_SHAPE", 3: "SVDQ_ERR_MISALIGNED",
@@ -84,9 +85,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_scales_to_canonical.argtypes, lib.svdq_scales_to_canonical.restype = [i64, i64, vp, vp, vp], st
     lib.svdq_check.argtypes, lib.svdq_check.restype = [vp], st
     lib.svdq_linear_quantize_next.argtypes = [Shape, vp, vp, vp, vp, vp, vp, ctypes.c_int32, vp, vp, vp, vp, vp, vp,
-                                              vp, sz, vp]
+                                              vp, sz, ctypes.c_uint, vp]
     lib.svdq_linear_quantize_next.restype = st
-    lib.svdq_linear_quantize_next_workspace.argtypes = [Shape, ctypes.c_int32, P(sz)]
+    lib.svdq_linear_quantize_next_workspace.argtypes = [Shape, ctypes.c_int32, ctypes.c_uint, P(sz)]
     lib.svdq_linear_quantize_next_workspace.restype = st
     lib.svdq_int4_act_sizes.argtypes, lib.svdq_int4_act_sizes.restype = [Shape, P(sz), P(sz), P(sz)], st
     lib.svdq_int4_weight_sizes.argtypes, lib.svdq_int4_weight_sizes.restype = [Shape, P(sz), P(sz)], st
@@ -215,15 +216,16 @@ def svdq_linear(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: P
     return Y
 
 
-def svdq_linear_quantize_next_workspace(shape: LayerShape, next_rank: int) -> int:
+def svdq_linear_quantize_next_workspace(shape: LayerShape, next_rank: int, flags: int = 0) -> int:
     v = ctypes.c_size_t()
-    _check(load().svdq_linear_quantize_next_workspace(shape.c(), next_rank, ctypes.byref(v)))
+    _check(load().svdq_linear_quantize_next_workspace(shape.c(), next_rank, flags, ctypes.byref(v)))
     return v.value
 
 
 def svdq_linear_quantize_next(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tensor | None, W: PreparedWeights,
                               next_inv_lambda: torch.Tensor, next_L1p: torch.Tensor | None, next_rank: int,
-                              store_y: bool = False, out: tuple | None = None, workspace: torch.Tensor | None = None):
+                              store_y: bool = False, out: tuple | None = None, workspace: torch.Tensor | None = None,
+                              flags: int = 0):
     """svdq_linear whose epilogue also quantizes Y for the next layer (K' = N).
     Returns (next_Qx [M][N/2] uint8, next_Sx native uint8, next_T [M][next_rank] bf16 or None,
     Y [M][N] bf16 or None)."""
@@ -239,12 +241,12 @@ def svdq_linear_quantize_next(Qx: torch.Tensor, Sx: torch.Tensor, T: torch.Tenso
         Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev) if store_y else None
     else:
         Qn, Sn, Tn, Y = out
-    need = svdq_linear_quantize_next_workspace(shape, next_rank)
+    need = svdq_linear_quantize_next_workspace(shape, next_rank, flags)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
     _check(load().svdq_linear_quantize_next(
         shape.c(), _ptr(Qx), _ptr(Sx), _ptr(T), _ptr(W.Qr), _ptr(W.Sr), _ptr(W.L2t), next_rank, _ptr(next_inv_lambda),
-        _ptr(next_L1p), _ptr(Qn), _ptr(Sn), _ptr(Tn), _ptr(Y), _ptr(workspace), workspace.numel(), _stream()))
+        _ptr(next_L1p), _ptr(Qn), _ptr(Sn), _ptr(Tn), _ptr(Y), _ptr(workspace), workspace.numel(), flags, _stream()))
     return Qn, Sn, Tn, Y
 
 
