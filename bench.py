@@ -103,7 +103,8 @@ def gemm_flops(w: synth.Workload) -> int:
     return 2 * w.M * w.N * w.K + 2 * w.M * w.rank * w.N
 
 
-GEMM_SOURCES = ("svdq_gemm.cuh", "svdq_gemm_pair.cuh", "svdq_gemm_common.cuh", "svdq_ptx.cuh")
+GEMM_SOURCES = ("svdq_gemm.cuh", "svdq_gemm_pair.cuh", "svdq_gemm_common.cuh", "svdq_gemm_qnext.cuh", "svdq_ptx.cuh",
+                "svdq_quant.cuh", "svdq_quant_tma.cuh")
 QUANT_SOURCES = ("svdq_quant_tma.cuh", "svdq_quant.cuh", "svdq_ptx.cuh")
 INT4_SOURCES = ("svdq_int4.cuh", "svdq_gemm_common.cuh", "svdq_ptx.cuh")
 
