@@ -732,6 +732,11 @@ def run_ours(args):
         # (the per-kernel pass above also pays each launch's latency)
         gemm_block_ms = timed_block(n_x, lambda i: S.svdq_linear(Qx, Sx, T if w.rank else None, sets[i % n_sets][1],
                                                                   S.SVDQ_FUSED, out=Y)) / n_x
+        # the quantizer alone, back to back on the rotating inputs (its launches
+        # overlap as in a network; no GEMM's dirty Y to write back between them)
+        quant_block_ms = timed_block(n_x, lambda i: S.svdq_quantize_act(
+            sets[i % n_sets][0], sets[i % n_sets][1].inv_lam, sets[i % n_sets][1].L1p, w.rank, w.N, S.SVDQ_FUSED,
+            out=(Qx, Sx, T))) / n_x
         lay = statistics.mean(step_ms)
         lay_f = statistics.mean(a + b for a, b in zip(k1f, k2f))
         q10, q50, q90 = np.percentile(step_ms, [10, 50, 90])
@@ -750,6 +755,9 @@ def run_ours(args):
             "gemm_block_ms": round(gemm_block_ms, 4),
             "gemm_block_frac": round(gemm_flops(w) / (gemm_block_ms * 1e-3) / 1e12 / fp4_peak, 4),
             "gemm_block_frac_datasheet_9pf": round(gemm_flops(w) / (gemm_block_ms * 1e-3) / 1e12 / DATASHEET_FP4_TFLOPS, 4),
+            "quantize_block_ms": round(quant_block_ms, 4),
+            "quantize_block_gbs": round(quantize_bytes(w) / (quant_block_ms * 1e-3) / 1e9, 1),
+            "quantize_block_frac_hbm": round(quantize_bytes(w) / (quant_block_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
             "bf16_cublas_ms": round(statistics.mean(kc), 4),
             "bf16_cublas_tflops": round(2 * w.M * w.N * w.K / (statistics.mean(kc) * 1e-3) / 1e12, 1),
         }
