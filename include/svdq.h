@@ -167,7 +167,8 @@ SVDQ_API svdq_status svdq_prepare_weights_static(svdq_shape shape, const void* W
  * Writes Qx codes [M][K/2], Sx native scales, T bf16 [M][rank]:
  *   x_hat = fp32(fp32(x) * inv_lambda[k]);
  *   per 16-group: s = E4M3_rne_satfinite(fp32(max|x_hat| / 6)),
- *                 q = E2M1_rne_satfinite(fp32(x_hat * fp32(1/s))), all +0 if s == 0;
+ *                 q = E2M1_rne_satfinite(x_hat / s) of the exact real quotient
+ *                     (ties to even), all +0 if s == 0;
  *   T = bf16(X L1p^T)  (fp32 accumulation)
  * (eq. (1), Table 3's NVFP4 microscaling, Fig. 6's fused down-projection).
  * variant SVDQ_FUSED reads X once; SVDQ_UNFUSED runs the down-projection as a
@@ -249,7 +250,8 @@ SVDQ_API svdq_status svdq_append_lowrank(svdq_shape shape, int32_t extra, const 
  * FP4 tensor cores: walkthrough eq. (1) with q_max = 2^(4-1) - 1 = 7; handbook,
  * Quantization chapter: one fp16 scale per 64 elements). Per 64-element group
  * along K:  s = fp16_rne(min(fp32(max|v| / 7), 65504)),
- *           q = clamp(rint(fp32(v * fp32(1/s))), -7, 7)  (all 0 when s == 0),
+ *           q = clamp(rint(v / s), -7, 7) of the exact real quotient (ties to
+ *               even; all 0 when s == 0),
  * and Y = bf16( sum_g sx[m,g] sw[n,g] sum_{k in g} qx[m,k] qr[n,k] + T L2 ).
  * Smoothing, L1p, L2t and T are those of the NVFP4 layer (svdq_prepare_weights);
  * only the residual and the activation are encoded differently.

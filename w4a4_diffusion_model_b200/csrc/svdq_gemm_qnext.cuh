@@ -60,22 +60,38 @@ __device__ __forceinline__ void epilogue_encode_next(const uint32_t (&p)[32 * BO
   static_assert(BOXES <= 2, "32 lanes x 4 factors cover 128 columns");
   const int row = row0 + lane;
   const int mpad = (M + 127) & ~127;
+  const float2 six = recip_bracket(6.0f);
 #pragma unroll
   for (int q = 0; q < BOXES; ++q) {   // four 16-groups (64 columns) at a time: one 32-bit word of scales
     uint32_t word = 0u;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int g = 4 * q + j;
-      float4 l[4];
+    for (int j = 0; j < 4; j += 2) {   // two groups at a time (their common path interleaves)
+      float4 l[2][4];
+      float2 v[2][8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k)   // factors 16g + 4k .. 16g + 4k + 3 sit in lane 4g + k
-        l[k] = make_float4(__shfl_sync(0xFFFFFFFFu, inv4.x, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.y, 4 * g + k),
-                           __shfl_sync(0xFFFFFFFFu, inv4.z, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.w, 4 * g + k));
-      uint2 codes;
-      uint32_t sb;
-      encode_group_vals(&p[8 * g], l, rcp_tbl, codes, sb);
-      if (row < M) *reinterpret_cast<uint2*>(nq.qx + (size_t)row * (size_t)(N >> 1) + ((col0 + 16 * g) >> 1)) = codes;
-      word |= sb << (8 * j);
+      for (int e = 0; e < 2; ++e) {
+        const int g = 4 * q + j + e;
+#pragma unroll
+        for (int k = 0; k < 4; ++k)   // factors 16g + 4k .. 16g + 4k + 3 sit in lane 4g + k
+          l[e][k] = make_float4(__shfl_sync(0xFFFFFFFFu, inv4.x, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.y, 4 * g + k),
+                                __shfl_sync(0xFFFFFFFFu, inv4.z, 4 * g + k), __shfl_sync(0xFFFFFFFFu, inv4.w, 4 * g + k));
+        smooth_group(&p[8 * g], l[e], v[e]);
+      }
+      uint2 codes[2];
+      uint32_t sb[2], bad = 0u;
+      encode_group_fast(v[0], six, rcp_tbl, codes[0], sb[0], bad);
+      encode_group_fast(v[1], six, rcp_tbl, codes[1], sb[1], bad);
+      if (bad != 0u) {   // a midpoint inside some bracket: the exact recipe
+        encode_group_vals(&p[8 * (4 * q + j)], l[0], rcp_tbl, codes[0], sb[0]);
+        encode_group_vals(&p[8 * (4 * q + j + 1)], l[1], rcp_tbl, codes[1], sb[1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int g = 4 * q + j + e;
+        if (row < M)
+          *reinterpret_cast<uint2*>(nq.qx + (size_t)row * (size_t)(N >> 1) + ((col0 + 16 * g) >> 1)) = codes[e];
+        word |= sb[e] << (8 * (j + e));
+      }
     }
     // rows past M carry zero accumulators, hence the zero scales of the padding rows
     if (row < mpad) *reinterpret_cast<uint32_t*>(nq.sx + native_scale_offset(row, (col0 >> 4) + 4 * q, N)) = word;

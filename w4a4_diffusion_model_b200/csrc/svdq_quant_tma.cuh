@@ -106,19 +106,24 @@ __device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
 }
 
 // The NVFP4 recipe of nvfp4_encode16 for one group given as 8 packed bf16
-// pairs and its 16 inverse smoothing factors (l[q] holds factors 4q..4q+3):
+// pairs and its 16 inverse smoothing factors (l[q] holds factors 4q..4q+3;
+// smooth_group forms the products v):
 //   v = fp32(x * inv_lambda); s = E4M3_rne_satfinite(fp32(max|v| / 6));
 //   q = E2M1_rne_satfinite(v / s) of the exact quotient, all +0 when s is 0.
 // The bracket (lo, hi) of 1/s comes from `rcp_tbl`, indexed by the E4M3 byte
 // of s (recip_bracket of its value).
-__device__ __forceinline__ void encode_group_vals(const uint32_t* w, const float4 (&l)[4], const float2* rcp_tbl,
-                                                  uint2& codes, uint32_t& sbyte) {
-  float2 v[8];
+__device__ __forceinline__ void smooth_group(const uint32_t* w, const float4 (&l)[4], float2 (&v)[8]) {
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
     v[2 * q] = mul2_rn(make_float2(bf16lo(w[2 * q]), bf16hi(w[2 * q])), make_float2(l[q].x, l[q].y));
     v[2 * q + 1] = mul2_rn(make_float2(bf16lo(w[2 * q + 1]), bf16hi(w[2 * q + 1])), make_float2(l[q].z, l[q].w));
   }
+}
+
+__device__ __forceinline__ void encode_group_vals(const uint32_t* w, const float4 (&l)[4], const float2* rcp_tbl,
+                                                  uint2& codes, uint32_t& sbyte) {
+  float2 v[8];
+  smooth_group(w, l, v);
   float m[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[i].x), fabsf(v[i].y));
@@ -159,9 +164,63 @@ __device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float
   encode_group_vals(w, l, rcp_tbl, codes, sbyte);
 }
 
-// Bracketing reciprocals of every E4M3 scale byte with the sign bit clear
-// (byte 0, a zero scale, is never looked up).
+// max(|a|, |b|, |c|).
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// E2M1 codes (round to nearest even, saturating) of 4 value pairs times f,
+// packed into one word: element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1_word(const float2* v, float f) {
+  const float2 p0 = mul2_rn(v[0], make_float2(f, f)), p1 = mul2_rn(v[1], make_float2(f, f));
+  const float2 p2 = mul2_rn(v[2], make_float2(f, f)), p3 = mul2_rn(v[3], make_float2(f, f));
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+  return r;
+}
+
+// The common path of encode_group_vals for one smoothed group v, without
+// branches (so that the two groups of a thread interleave):
+//   scale byte: amax times the bracket (lo, hi) of 1/6, both products
+//   converted by one cvt; they give the same byte unless an E4M3 midpoint (or
+//   the saturation bound) lies strictly between them, and then that byte is
+//   the exact one (rounding is monotone);
+//   codes: both bracket products of 1/s, from the table (e4m3_recip_bracket).
+// `bad` is set when a pair disagrees; the caller then redoes the group with
+// encode_group_vals (IEEE quotient for the scale, exact fix-up of the codes).
+// A zero scale gives all +0 codes.
+__device__ __forceinline__ void encode_group_fast(const float2 (&v)[8], float2 six, const float2* rcp_tbl,
+                                                  uint2& codes, uint32_t& sbyte, uint32_t& bad) {
+  const float m0 = max3_abs(v[0].x, v[0].y, v[1].x), m1 = max3_abs(v[1].y, v[2].x, v[2].y);
+  const float m2 = max3_abs(v[3].x, v[3].y, v[4].x), m3 = max3_abs(v[4].y, v[5].x, v[5].y);
+  const float m4 = max3_abs(v[6].x, v[6].y, v[7].x);
+  const float amax = fmaxf(max3_abs(m0, m1, m2), max3_abs(m3, m4, v[7].y));
+  const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(mul2_rn(make_float2(amax, amax), six), __NV_SATFINITE,
+                                                          __NV_E4M3);
+  const uint32_t b = two & 0xFFu;
+  const float2 ib = rcp_tbl[b & 0x7Fu];
+  const uint32_t l0 = e2m1_word(v, ib.x), l1 = e2m1_word(v + 4, ib.x);
+  const uint32_t h0 = e2m1_word(v, ib.y), h1 = e2m1_word(v + 4, ib.y);
+  bad |= ((two >> 8) ^ b) | (l0 ^ h0) | (l1 ^ h1);
+  codes = b != 0u ? make_uint2(l0, l1) : make_uint2(0u, 0u);
+  sbyte = b;
+}
+
+// Entry `byte` of the table of bracketing reciprocals indexed by an E4M3
+// scale byte with the sign bit clear: recip_bracket of its value, and (0, 0)
+// for byte 0 (a zero scale: encode_group_fast multiplies by zero and selects
+// +0 codes; encode_group_vals never looks it up).
 __device__ __forceinline__ float2 e4m3_recip_bracket(uint32_t byte) {
+  if (byte == 0u) return make_float2(0.f, 0.f);
   const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
   return recip_bracket(sv);
 }
@@ -329,6 +388,12 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
     const int rA = m0 + rl, rB = rA + 8;
     const bool okA = rA < M, okB = rB < M;
     const size_t ldq = (size_t)K >> 1;
+    const int cfirst = st0 * L::kCols + 64 * h + 16 * t;   // first column of this thread's group in stage 0
+    uint8_t* qpa = Qx + (size_t)rA * ldq + (cfirst >> 1);
+    uint8_t* qpb = Qx + (size_t)rB * ldq + (cfirst >> 1);
+    uint8_t* spa = Sx + native_scale_offset(rA, cfirst >> 4, K);
+    uint8_t* spb = Sx + native_scale_offset(rB, cfirst >> 4, K);
+    const float2 six = recip_bracket(6.0f);
     for (int j = 0; j < nst; ++j) {
       const int s = j % L::kStages;
       if (!mbar_wait(full + s, (j / L::kStages) & 1u, kDevErrTimeoutFull)) break;
@@ -345,9 +410,9 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
         xb[0] = b0.x; xb[1] = b0.y; xb[2] = b0.z; xb[3] = b0.w;
         xb[4] = b1.x; xb[5] = b1.y; xb[6] = b1.z; xb[7] = b1.w;
       }
-      const int c = (st0 + j) * L::kCols + 64 * h + 16 * t;   // first column of this thread's group
       const float* il = reinterpret_cast<const float*>(st + kQStageXBytes + L::kL1) + 64 * h + 16 * t;
       if constexpr (CODEC == kCodecInt4) {
+        const int c = (st0 + j) * L::kCols + 64 * h + 16 * t;   // first column of this thread's group
         uint4 qa, qb;
         float sA, sB;
         encode_int4_quarter(xa, il, qa, sA);
@@ -361,26 +426,33 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
           S[rA] = sA;
           S[rB] = sB;
         }
-        continue;
-      }
-      uint2 qa, qb;
-      uint32_t sbA, sbB;
-      encode_group_bf16(xa, il, rcp_tbl, qa, sbA);
-      encode_group_bf16(xb, il, rcp_tbl, qb, sbB);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty + s);         // the stage's shared memory is no longer read
-      if (okA) *reinterpret_cast<uint2*>(Qx + (size_t)rA * ldq + (c >> 1)) = qa;
-      if (okB) *reinterpret_cast<uint2*>(Qx + (size_t)rB * ldq + (c >> 1)) = qb;
-      // the four scale bytes of a row and slab are adjacent in the native layout
-      const uint32_t a1 = __shfl_down_sync(0xFFFFFFFFu, sbA, 1), a2 = __shfl_down_sync(0xFFFFFFFFu, sbA, 2),
-                     a3 = __shfl_down_sync(0xFFFFFFFFu, sbA, 3);
-      const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, sbB, 1), b2 = __shfl_down_sync(0xFFFFFFFFu, sbB, 2),
-                     b3 = __shfl_down_sync(0xFFFFFFFFu, sbB, 3);
-      if (t == 0) {   // rows past M get zero scales: TMA zero-fills them
-        *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rA, c >> 4, K)) =
-            sbA | (a1 << 8) | (a2 << 16) | (a3 << 24);
-        *reinterpret_cast<uint32_t*>(Sx + native_scale_offset(rB, c >> 4, K)) =
-            sbB | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      } else {
+        float4 l[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) l[q] = *reinterpret_cast<const float4*>(il + 4 * q);
+        // The stage's shared memory has been read into registers: release it
+        // before encoding (the arrive's release semantics order the loads
+        // before it), so that its refill overlaps the work below.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + s);
+        float2 va[8], vb[8];
+        smooth_group(xa, l, va);
+        smooth_group(xb, l, vb);
+        uint2 qa, qb;
+        uint32_t sbA, sbB, bad = 0u;
+        encode_group_fast(va, six, rcp_tbl, qa, sbA, bad);
+        encode_group_fast(vb, six, rcp_tbl, qb, sbB, bad);
+        if (bad != 0u) {   // a midpoint inside some bracket: the exact recipe for both groups
+          encode_group_vals(xa, l, rcp_tbl, qa, sbA);
+          encode_group_vals(xb, l, rcp_tbl, qb, sbB);
+        }
+        if (okA) *reinterpret_cast<uint2*>(qpa) = qa;
+        if (okB) *reinterpret_cast<uint2*>(qpb) = qb;
+        // rows past M get zero scales: TMA zero-fills them
+        *spa = (uint8_t)sbA;
+        *spb = (uint8_t)sbB;
+        qpa += L::kCols / 2; qpb += L::kCols / 2;
+        spa += (L::kCols / 64) * 512; spb += (L::kCols / 64) * 512;
       }
     }
   }
