@@ -25,6 +25,43 @@ __host__ __device__ __forceinline__ size_t native_scale_offset(int r, int g, int
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Two IEEE round-to-nearest fp32 products in one instruction.
+__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\t"
+      "mov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// max(|a|, |b|, |c|).
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// E2M1 codes (round to nearest even, saturating) of 4 value pairs times f,
+// packed into one word: element 2i in the low nibble of byte i.
+__device__ __forceinline__ uint32_t e2m1_word(const float2* v, float f) {
+  const float2 p0 = mul2_rn(v[0], make_float2(f, f)), p1 = mul2_rn(v[1], make_float2(f, f));
+  const float2 p2 = mul2_rn(v[2], make_float2(f, f)), p3 = mul2_rn(v[3], make_float2(f, f));
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
+  return r;
+}
+
 // ---------------------------------------------------------------- exact-quotient rounding
 // The codes are round-to-nearest-even images of the EXACT quotient v / s
 // (walkthrough eq. (1): round(X / s)). Multiplying by one rounded reciprocal
@@ -43,6 +80,16 @@ __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w &
 __device__ __forceinline__ float2 recip_bracket(float s) {
   const float r = __frcp_rn(s);
   return make_float2(__fmul_rn(r, 1.0f - 0x1p-21f), __fmul_rn(r, 1.0f + 0x1p-21f));
+}
+
+// Entry `byte` of the table of bracketing reciprocals indexed by an E4M3
+// scale byte with the sign bit clear: recip_bracket of its value, and (0, 0)
+// for byte 0 (a zero scale: encode_group_fast multiplies by zero and selects
+// +0 codes; encode_group_vals never looks it up).
+__device__ __forceinline__ float2 e4m3_recip_bracket(uint32_t byte) {
+  if (byte == 0u) return make_float2(0.f, 0.f);
+  const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
+  return recip_bracket(sv);
 }
 
 // The exact code of v / s, given the code a of the lower bracket product
@@ -113,34 +160,49 @@ __device__ __forceinline__ void nvfp4_encode16(const float (&v)[16], uint2& code
 }
 
 // The same NVFP4 recipe for a group of 16 held by two lanes (lane ^ 1), 8
-// values each: the group's amax is pooled with one shuffle, both lanes derive
-// the same scale, and each lane returns the packed codes of its own 8 values
-// (one 32-bit word: element 2i in the low nibble of byte i). Every lane of the
-// warp must call it.
-__device__ __forceinline__ void nvfp4_encode8_pair(const float (&v)[8], uint32_t& codes, uint32_t& sbyte) {
-  float amax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-  amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, 1));
-  const __nv_fp8_storage_t sb = __nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
-  const float sval = __half2float(__half(__nv_cvt_fp8_to_halfraw(sb, __NV_E4M3)));
-  sbyte = (uint32_t)sb;
-  if (sval == 0.f) {
-    codes = 0u;
-    return;
+// values each (element 2i in d[i].x, 2i+1 in d[i].y): the group's amax is
+// pooled with one shuffle, both lanes derive the same scale, and each lane
+// returns the packed codes of its own 8 values (one 32-bit word: element j in
+// nibble j). Made for inputs on which exact midpoint ties are common (the
+// DeltaQuant deltas: a bf16 token minus an E4M3 core, divided by an E4M3
+// scale, lands on a midpoint for ~2 % of elements):
+//   scale byte: amax times the bracket of 1/6, both products converted by one
+//   cvt; the IEEE quotient only where the two bytes differ;
+//   codes: both bracket products of 1/s (rcp_tbl: e4m3_recip_bracket per byte);
+//   each nibble where they differ is resolved on its own by e2m1_exact_nibble,
+//   looping over the differing nibbles only.
+// Every lane of the warp must call it.
+__device__ __forceinline__ void nvfp4_encode8_pair(const float2 (&d)[4], const float2* rcp_tbl, float2 six,
+                                                   uint32_t& codes, uint32_t& sbyte) {
+  const float m = fmaxf(max3_abs(d[0].x, d[0].y, d[1].x), max3_abs(d[1].y, d[2].x, max3_abs(d[2].y, d[3].x, d[3].y)));
+  const float amax = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+  const uint32_t two = (uint32_t)__nv_cvt_float2_to_fp8x2(mul2_rn(make_float2(amax, amax), six), __NV_SATFINITE,
+                                                          __NV_E4M3);
+  uint32_t b = two & 0xFFu;
+  if ((two >> 8) != b) b = (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(amax, 6.0f), __NV_SATFINITE, __NV_E4M3);
+  sbyte = b;
+  const float2 ib = rcp_tbl[b & 0x7Fu];
+  uint32_t lo = e2m1_word(d, ib.x);
+  uint32_t diff = lo ^ e2m1_word(d, ib.y);
+  if (diff != 0u) {
+    const float s4 = 0.25f * __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3)));
+    do {
+      const int j = (__ffs((int)diff) - 1) >> 2;     // the lowest differing element
+      float v = d[0].x;
+      v = j == 1 ? d[0].y : v;
+      v = j == 2 ? d[1].x : v;
+      v = j == 3 ? d[1].y : v;
+      v = j == 4 ? d[2].x : v;
+      v = j == 5 ? d[2].y : v;
+      v = j == 6 ? d[3].x : v;
+      v = j == 7 ? d[3].y : v;
+      const uint32_t sh = 4u * (uint32_t)j;
+      const uint32_t nib = e2m1_exact_nibble(v, s4, (lo >> sh) & 0xFu);
+      lo = (lo & ~(0xFu << sh)) | (nib << sh);
+      diff &= ~(0xFu << sh);
+    } while (diff != 0u);
   }
-  const float2 ib = recip_bracket(sval);
-  uint32_t lo = 0u, hi = 0u;
-  float2 p[8];
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    p[b] = make_float2(v[2 * b], v[2 * b + 1]);
-    lo |= e2m1_pair(p[b], ib.x) << (8 * b);
-    hi |= e2m1_pair(p[b], ib.y) << (8 * b);
-  }
-#pragma unroll
-  for (int b = 4; b < 8; ++b) p[b] = make_float2(0.f, 0.f);
-  codes = e2m1_group_exact(p, sval, make_uint2(lo, 0u), make_uint2(hi, 0u)).x;
+  codes = b != 0u ? lo : 0u;
 }
 
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,

@@ -92,19 +92,6 @@ __device__ __forceinline__ void tma_load_2d_once(void* dst, const void* tmap, ui
 // Byte offset of 16-byte chunk c of row r in a 128B-swizzled box (128-byte rows).
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4)); }
 
-// Two IEEE round-to-nearest fp32 products in one instruction.
-__device__ __forceinline__ float2 mul2_rn(float2 a, float2 b) {
-  float2 d;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\t"
-      "mov.b64 rb, {%4, %5};\n\t"
-      "mul.rn.f32x2 rd, ra, rb;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
-
 // The NVFP4 recipe of nvfp4_encode16 for one group given as 8 packed bf16
 // pairs and its 16 inverse smoothing factors (l[q] holds factors 4q..4q+3;
 // smooth_group forms the products v):
@@ -164,30 +151,6 @@ __device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float
   encode_group_vals(w, l, rcp_tbl, codes, sbyte);
 }
 
-// max(|a|, |b|, |c|).
-__device__ __forceinline__ float max3_abs(float a, float b, float c) {
-  float d;
-  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
-}
-
-// E2M1 codes (round to nearest even, saturating) of 4 value pairs times f,
-// packed into one word: element 2i in the low nibble of byte i.
-__device__ __forceinline__ uint32_t e2m1_word(const float2* v, float f) {
-  const float2 p0 = mul2_rn(v[0], make_float2(f, f)), p1 = mul2_rn(v[1], make_float2(f, f));
-  const float2 p2 = mul2_rn(v[2], make_float2(f, f)), p3 = mul2_rn(v[3], make_float2(f, f));
-  uint32_t r;
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
-      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
-      : "=r"(r)
-      : "f"(p0.x), "f"(p0.y), "f"(p1.x), "f"(p1.y), "f"(p2.x), "f"(p2.y), "f"(p3.x), "f"(p3.y));
-  return r;
-}
-
 // The common path of encode_group_vals for one smoothed group v, without
 // branches (so that the two groups of a thread interleave):
 //   scale byte: amax times the bracket (lo, hi) of 1/6, both products
@@ -213,16 +176,6 @@ __device__ __forceinline__ void encode_group_fast(const float2 (&v)[8], float2 s
   bad |= ((two >> 8) ^ b) | (l0 ^ h0) | (l1 ^ h1);
   codes = b != 0u ? make_uint2(l0, l1) : make_uint2(0u, 0u);
   sbyte = b;
-}
-
-// Entry `byte` of the table of bracketing reciprocals indexed by an E4M3
-// scale byte with the sign bit clear: recip_bracket of its value, and (0, 0)
-// for byte 0 (a zero scale: encode_group_fast multiplies by zero and selects
-// +0 codes; encode_group_vals never looks it up).
-__device__ __forceinline__ float2 e4m3_recip_bracket(uint32_t byte) {
-  if (byte == 0u) return make_float2(0.f, 0.f);
-  const float sv = __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
-  return recip_bracket(sv);
 }
 
 // What the quantizing warps produce besides T.
