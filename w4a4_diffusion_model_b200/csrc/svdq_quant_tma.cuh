@@ -283,6 +283,10 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
   }
+  if (warp == L::kProducerWarp && lane == 0) {   // descriptors are kernel parameters: no dependency
+    prefetch_tmap(&tm_x);
+    if (RANK > 0) prefetch_tmap(&tm_l1);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -293,8 +297,6 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
   if (warp == L::kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tmap(&tm_x);
-      if (RANK > 0) prefetch_tmap(&tm_l1);
       for (int j = 0; j < nst; ++j) {
         const int s = j % L::kStages;
         if (!mbar_wait(empty + s, ((j / L::kStages) & 1u) ^ 1u, kDevErrTimeoutEmpty)) break;
