@@ -148,7 +148,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
         // Another role gave up: let the copies this thread issued land before
         // the CTA exits (bounded; only the last STAGES stages can be in flight).
         for (uint32_t j = it > (uint32_t)STAGES ? it - STAGES : 0u; j < it; ++j)
-          mbar_wait(full + j % STAGES, (j / STAGES) & 1u, kDevErrTimeoutFull);
+          mbar_drain(full + j % STAGES, (j / STAGES) & 1u);
       }
     }
   } else if (warp >= kSfWarp0) {
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_kernel(
       if (!ok) {
         // Gave up: wait (bounded) for the MMAs already issued before TMEM is freed.
         tc_commit(mma_drain);
-        mbar_wait(mma_drain, 0, kDevErrTimeoutAccum);
+        mbar_drain(mma_drain, 0);
       }
     }
   } else {

@@ -220,11 +220,11 @@ __device__ __forceinline__ void epilogue_next_lowrank(
   }
   // leave no TMA load of L1p' in flight (the last one was consumed already
   // unless the loop stopped early; waiting on a completed phase returns at once)
-  if (loader && l1_issued > 0) mbar_wait(l1_full + h, (l1_issued - 1u) & 1u, kDevErrTimeoutNext);
+  if (loader && l1_issued > 0) mbar_drain(l1_full + h, (l1_issued - 1u) & 1u);
   // and no T' MMA running when TMEM is freed
   if (issuer && tcount + (ok ? 0u : 1u) > 0) {
     tc_commit_pair(tp_drain, 0x1);
-    mbar_wait(tp_drain, 0, kDevErrTimeoutNext);
+    mbar_drain(tp_drain, 0);
   }
 }
 
@@ -367,9 +367,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
           }
         }
       }
-      if (device_error_set()) {
+      if (device_error_set()) {   // let the copies this thread issued land before the CTA exits
         for (uint32_t j = it > (uint32_t)STAGES ? it - STAGES : 0u; j < it; ++j)
-          mbar_wait(full + j % STAGES, (j / STAGES) & 1u, kDevErrTimeoutFull);
+          mbar_drain(full + j % STAGES, (j / STAGES) & 1u);
       }
     }
   } else if (warp >= kSfWarp0) {
@@ -495,7 +495,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) svdq_gemm_pair_kernel(
       }
       if (!ok) {
         tc_commit_pair(mma_drain, 0x1);
-        mbar_wait(mma_drain, 0, kDevErrTimeoutAccum);
+        mbar_drain(mma_drain, 0);
       }
     }
   } else {

@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
         // Another role gave up: let the copies this thread issued land before
         // the CTA exits (bounded; only the last kI4Stages stages can be in flight).
         for (uint32_t j = it > (uint32_t)kI4Stages ? it - kI4Stages : 0u; j < it; ++j)
-          mbar_wait(full + j % kI4Stages, (j / kI4Stages) & 1u, kDevErrTimeoutFull);
+          mbar_drain(full + j % kI4Stages, (j / kI4Stages) & 1u);
       }
     }
   } else if (warp == kI4MmaWarp) {
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kI4Threads, 1) svdq_int4_gemm_kernel(
       if (!ok) {
         // Gave up: wait (bounded) for the MMAs already issued before TMEM is freed.
         tc_commit(mma_drain);
-        mbar_wait(mma_drain, 0, kDevErrTimeoutAccum);
+        mbar_drain(mma_drain, 0);
       }
     }
   } else {

@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
   if (warp == L::kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
-      for (int j = 0; j < nst; ++j) {
+      int j = 0;
+      for (; j < nst; ++j) {
         const int s = j % L::kStages;
         if (!mbar_wait(empty + s, ((j / L::kStages) & 1u) ^ 1u, kDevErrTimeoutEmpty)) break;
         unsigned char* st = smem + s * L::kStage;
@@ -309,6 +310,10 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
           if (RANK > 0) tma_load_2d(st + kQStageXBytes + b * L::kL1Box, &tm_l1, full + s, c0 + 64 * b, 0);
         }
         if (QUANT) bulk_load(st + kQStageXBytes + L::kL1, inv_lambda + c0, (uint32_t)L::kInv, full + s);
+      }
+      if (device_error_set()) {   // let the copies issued land before the CTA exits
+        for (int i = j > L::kStages ? j - L::kStages : 0; i < j; ++i)
+          mbar_drain(full + i % L::kStages, (uint32_t)(i / L::kStages) & 1u);
       }
     }
   } else if (warp == L::kMmaWarp) {
@@ -461,6 +466,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
       tc_fence_before();
       if (ksplit > 1) cluster_sync(); else __syncthreads();   // pushes visible; TMEM reads done
       if (warp == L::kMmaWarp) {
+        mbar_drain(acc_bar, 0u);   // every down-projection MMA has completed (also after a failure)
         tc_fence_after();
         tmem_dealloc(tmem, L::kTmemCols);
       }
@@ -519,6 +525,7 @@ __global__ void __launch_bounds__(QuantSmem<RANK, BM>::kThreads, 1) quantize_tma
       tc_fence_before();
       __syncthreads();
       if (warp == L::kMmaWarp) {
+        mbar_drain(acc_bar, 0u);   // every down-projection MMA has completed (also after a failure)
         tc_fence_after();
         tmem_dealloc(tmem, L::kTmemCols);
       }
