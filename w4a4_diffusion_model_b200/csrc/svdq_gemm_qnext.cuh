@@ -8,8 +8,10 @@
 //
 // Per epilogue warp (32 rows x 64*BOXES columns of one tile, row = lane), each
 // thread encodes its row's 16-element groups from the packed bf16 registers
-// with the quantizer's own recipe (encode_group_bf16: x_hat = fp32(y * inv'),
-// E4M3 scale of max|x_hat| / 6, E2M1 codes of x_hat / s), writes the packed
+// with the quantizer's own recipe (smooth_group: x_hat = fp32(y * inv'); then
+// encode_group_fast, two groups at a time, and encode_group_vals where a
+// bracket straddles a midpoint: E4M3 scale of max|x_hat| / 6, E2M1 codes of
+// x_hat / s, both of the exact quotients), writes the packed
 // codes and the scale bytes in the native tile layout, and stores its band of
 // Y (TMA, as the plain epilogue does) only when the caller asked for Y.
 //

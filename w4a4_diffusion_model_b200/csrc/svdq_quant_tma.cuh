@@ -142,15 +142,6 @@ __device__ __forceinline__ void encode_group_vals(const uint32_t* w, const float
   codes = e2m1_group_exact(v, sval, make_uint2(lo[0], lo[1]), make_uint2(hi[0], hi[1]));
 }
 
-// The same with the 16 inverse smoothing factors read from `il` (any space).
-__device__ __forceinline__ void encode_group_bf16(const uint32_t* w, const float* il, const float2* rcp_tbl,
-                                                  uint2& codes, uint32_t& sbyte) {
-  float4 l[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) l[q] = *reinterpret_cast<const float4*>(il + 4 * q);
-  encode_group_vals(w, l, rcp_tbl, codes, sbyte);
-}
-
 // The common path of encode_group_vals for one smoothed group v, without
 // branches (so that the two groups of a thread interleave):
 //   scale byte: amax times the bracket (lo, hi) of 1/6, both products
