@@ -46,6 +46,38 @@ __device__ __forceinline__ float e4m3_to_float(uint32_t byte) {
   return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)byte, __NV_E4M3)));
 }
 
+// The two bf16 values of w (low half first) plus, or minus, fp32 operands:
+// exact conversions, one round-to-nearest-even each (mixed-precision
+// add / sub with the bf16 operand first).
+__device__ __forceinline__ float2 bf16x2_add_f32(uint32_t w, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "add.rn.f32.bf16 %0, l, %3;\n\tadd.rn.f32.bf16 %1, h, %4;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "r"(w), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 bf16x2_sub_f32(uint32_t w, float c0, float c1) {
+  float2 r;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "sub.rn.f32.bf16 %0, l, %3;\n\tsub.rn.f32.bf16 %1, h, %4;\n\t}"
+      : "=f"(r.x), "=f"(r.y) : "r"(w), "f"(c0), "f"(c1));
+  return r;
+}
+
+// Per 16-bit half: max and min of unsigned values.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+
 constexpr int kDqThreads = 128;
 constexpr int kDqGroupsPerCta = kDqThreads / 2;
 // Five CTAs per SM (96 registers a thread): the kernel is bound by issue
@@ -93,35 +125,39 @@ __global__ void __launch_bounds__(kDqThreads, 5) deltaquant_encode_kernel(const 
     xw[4 * t + 0] = a.x; xw[4 * t + 1] = a.y; xw[4 * t + 2] = a.z; xw[4 * t + 3] = a.w;
   }
   // fp32 sums (exact when the spread test below passes), |x| max and nonzero
-  // |x| min per channel; missing tokens hold +0 and change none of them
-  float sum[8], mx[8];
-  uint32_t mn[8];
+  // |x| min per channel, the last two on the bf16 bit patterns of a channel
+  // pair at once (magnitudes order like their patterns; a zero becomes 0x7FFF
+  // through a borrow-free per-half decrement, above every finite magnitude
+  // minus one); missing tokens hold +0 and change none of them
+  float2 sum[4];
+  uint32_t mx2[4], mn2[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sum[i] = 0.f;
-    mx[i] = 0.f;
-    mn[i] = 0xFFFFFFFFu;
+  for (int i = 0; i < 4; ++i) {
+    sum[i] = make_float2(0.f, 0.f);
+    mx2[i] = 0u;
+    mn2[i] = 0x7FFF7FFFu;
   }
 #pragma unroll
   for (int t = 0; t < 8; ++t)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const uint32_t w = xw[4 * t + (i >> 1)];
-      const uint32_t u = (i & 1) ? (w & 0xFFFF0000u) : (w << 16);
-      sum[i] = __fadd_rn(sum[i], __uint_as_float(u));
-      mx[i] = fmaxf(mx[i], fabsf(__uint_as_float(u)));
-      mn[i] = min(mn[i], (u & 0x7FFFFFFFu) - 1u);         // a zero wraps to the maximum
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t w = xw[4 * t + i];
+      sum[i] = bf16x2_add_f32(w, sum[i]);
+      mx2[i] = max_u16x2(mx2[i], w & 0x7FFF7FFFu);
+      mn2[i] = min_u16x2(mn2[i], ((w | 0x80008000u) - 0x00010001u) & 0x7FFF7FFFu);
     }
   const float inv_n = 1.0f / (float)n;                    // n is 1, 2, 4 or 8: exact
   float cval[8];
   uint32_t cb[2] = {0u, 0u};
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const float mnf = __uint_as_float(mn[i] + 1u);        // +0 when every value is zero
-    const bool exact = mx[i] < 0x1p124f && (mn[i] == 0xFFFFFFFFu || mx[i] <= mnf * 8192.0f);
+    const uint32_t mxb = (mx2[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;   // max |x|, bf16 bits
+    const uint32_t mnz = (mn2[i >> 1] >> (16 * (i & 1))) & 0xFFFFu;   // min nonzero |x| bits - 1, 0x7FFF: none
+    const float mxf = __uint_as_float(mxb << 16), mnf = __uint_as_float((mnz + 1u) << 16);
+    const bool exact = mxb < 0x7D80u && (mnz == 0x7FFFu || mxf <= mnf * 8192.0f);   // 0x7D80: 2^124
     uint32_t byte;
     if (exact) {
-      const float mean = sum[i] * inv_n;
+      const float mean = ((i & 1) ? sum[i >> 1].y : sum[i >> 1].x) * inv_n;
       byte = mean == 0.f ? 0u : (uint32_t)__nv_cvt_float_to_fp8(mean, __NV_SATFINITE, __NV_E4M3);
     } else {   // wide range: the fp64 sum in token order (i and t are compile-time: registers only)
       double sd = 0.0;
@@ -148,10 +184,7 @@ __global__ void __launch_bounds__(kDqThreads, 5) deltaquant_encode_kernel(const 
   for (int t = 0; t < 8; ++t) {
     float2 d[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t w = xw[4 * t + i];
-      d[i] = make_float2(__fsub_rn(bf16lo(w), cval[2 * i]), __fsub_rn(bf16hi(w), cval[2 * i + 1]));
-    }
+    for (int i = 0; i < 4; ++i) d[i] = bf16x2_sub_f32(xw[4 * t + i], cval[2 * i], cval[2 * i + 1]);
     uint32_t codes, sb;
     nvfp4_encode8_pair(d, rcp_tbl, six, codes, sb);
     // lanes 8j, 8j+2, 8j+4, 8j+6 hold the scales of groups 4j'..4j'+3
