@@ -80,11 +80,11 @@ __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
 
 constexpr int kDqThreads = 128;
 constexpr int kDqGroupsPerCta = kDqThreads / 2;
-// Five CTAs per SM (96 registers a thread): the kernel is bound by issue
-// latency, and 20 resident warps hide more of it than 16 (measured 1792 against
-// 1680 GB/s; six CTAs spill and run at 1725 GB/s).
+// Six CTAs per SM (80 registers a thread, no spill): the kernel is bound by
+// issue latency, and more resident warps hide more of it (measured 1880
+// against 1851 GB/s at five CTAs; seven and eight spill and run at ~1860).
 
-__global__ void __launch_bounds__(kDqThreads, 5) deltaquant_encode_kernel(const __nv_bfloat16* __restrict__ X,
+__global__ void __launch_bounds__(kDqThreads, 6) deltaquant_encode_kernel(const __nv_bfloat16* __restrict__ X,
                                                                        uint8_t* __restrict__ core,
                                                                        uint8_t* __restrict__ Qd,
                                                                        uint8_t* __restrict__ Sd, int F, int H, int W,
