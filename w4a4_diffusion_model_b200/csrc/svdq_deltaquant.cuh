@@ -80,7 +80,7 @@ __device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
 
 constexpr int kDqThreads = 128;
 constexpr int kDqGroupsPerCta = kDqThreads / 2;
-// Six CTAs per SM (80 registers a thread, no spill): the kernel is bound by
+// Six CTAs per SM (79 registers a thread, no spill): the kernel is bound by
 // issue latency, and more resident warps hide more of it (measured 1880
 // against 1851 GB/s at five CTAs; seven and eight spill and run at ~1860).
 
