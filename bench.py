@@ -450,6 +450,18 @@ def flux_shape_summary(S, w: synth.Workload, dev, n: int, fp4_peak: float) -> di
             "fp4_peak_tflops": round(fp4_peak, 1), "input_sets": n_sets}
 
 
+def scale_group_stats(S, native, rows: int, K: int) -> dict:
+    """Counts over the E4M3 group scales of a native scale buffer (rows x K/16
+    groups): zero (an all-zero group, or amax / 6 below half the smallest
+    subnormal: every code +0), subnormal (exponent field 0: fewer significant
+    bits in the scale) and saturated (448, the largest finite E4M3 value: the
+    group's amax / 6 reached it and its largest values may clip)."""
+    c = S.svdq_scales_to_canonical(native, rows, K)
+    zero = int((c == 0).sum())
+    return {"groups": int(c.numel()), "zero": zero, "subnormal": int(((c & 0x78) == 0).sum()) - zero,
+            "saturated": int((c == 0x7E).sum())}
+
+
 def deltaquant_bytes(F: int, H: int, W: int, C: int) -> int:
     """Algorithmic HBM bytes of one DeltaQuant encode: read the bf16 tokens;
     write the E4M3 cores, the packed delta codes and their native scales."""
@@ -793,6 +805,12 @@ def run_ours(args):
         # the other FLUX projections, where the GEMM target is stated
         extras["other_flux_shapes"] = [flux_shape_summary(S, o, dev, n_x, fp4_peak)
                                        for o in (synth.FLUX_MLP_UP, synth.FLUX_MLP_DOWN) if o.name != w.name]
+
+        # how the workload's groups sit in the E4M3 scale range (activations of
+        # one step, the prepared weights)
+        S.svdq_quantize_act(X, P.inv_lam, P.L1p, w.rank, w.N, S.SVDQ_FUSED, out=(Qx, Sx, T))
+        extras["scale_groups"] = {"activations": scale_group_stats(S, Sx, w.M, w.K),
+                                  "weights": scale_group_stats(S, P.Sr, w.N, w.K)}
 
         extras["deltaquant"] = deltaquant_summary(S, dev, n_x)
         extras["deltaquant"]["frac_hbm"] = round(extras["deltaquant"]["gbs"] / peaks["hbm_gbs"], 4)

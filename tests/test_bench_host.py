@@ -146,3 +146,15 @@ def test_int4_quantize_bytes():
     assert bench.quantize_bytes_int4(w) == (2 * 4608 * 3072 + 4 * 3072 + 2 * 32 * 3072 + 4608 * 3072
                                             + 4608 * 48 * 4 + 2 * 4608 * 32)
     assert bench.quantize_bytes_int4(w.with_(M=130)) - bench.quantize_bytes_int4(w.with_(M=129)) == 2 * 3072 + 3072 + 64
+
+
+def test_scale_group_stats_classes():
+    """E4M3 scale bytes: 0 (zero / underflow), exponent field 0 with a nonzero
+    mantissa (subnormal), 0x7E (448, saturated), the rest normal."""
+    class FakeS:
+        @staticmethod
+        def svdq_scales_to_canonical(native, rows, K):
+            return native.view(rows, K // 16)
+    b = torch.tensor([[0x00, 0x01, 0x07, 0x08, 0x38, 0x7E, 0x7E, 0x00]], dtype=torch.uint8)
+    st = bench.scale_group_stats(FakeS, b, 1, 128)
+    assert st == {"groups": 8, "zero": 2, "subnormal": 2, "saturated": 2}
