@@ -64,6 +64,8 @@ def parse():
     p.add_argument("--no-extras", action="store_true", help="skip the cuBLAS / unfused / rank-0 / e2e / CPU legs")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     p.add_argument("--extra-json", default=None, help="append per-leg details to this JSONL file")
+    p.add_argument("--deltaquant-only", action="store_true",
+                   help="time only the DeltaQuant encoder on the bench's video latent (one JSON line; for profiling)")
     return p.parse_args()
 
 
@@ -916,10 +918,23 @@ def run_ours(args):
     return 0
 
 
+def run_deltaquant_only(args) -> int:
+    """The DeltaQuant encoder alone on one GPU (a few launches, no other kernel)."""
+    from w4a4_diffusion_model_b200 import svdq as S
+    if not torch.cuda.is_available():
+        raise RuntimeError("the DeltaQuant encoder needs a CUDA device (there is no CPU fallback)")
+    S.load()
+    dev = torch.device("cuda", 0)
+    print(json.dumps(deltaquant_summary(S, dev, max(1, args.steps))), flush=True)
+    return 0
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.deltaquant_only:
+        return run_deltaquant_only(args)
     return run_ours(args)
 
 
